@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the ARL2 hybrid attention layer on B200.
+
+One step = the full 21-frame forward of the Wan-1.3B-shaped 480p layer
+(B=1, H=12, d=128, 21 latent frames x 1560 tokens, bf16 I/O, fp32 state,
+one clean pass per frame): the state is reset to S_0 = 0 and every frame runs
+attention, the inter-frame read and the gated delta update through the C ABI.
+Inputs of all 21 frames (302 MB of q/k/v, larger than the 126 MB L2) are
+resident in HBM before timing, so consecutive frames and steps do not hit in
+L2 on their inputs.
+
+``value`` is tokens/s over the whole job (every rank's frames / max over ranks
+of the device time); ``e2e`` is the same metric with each step's inputs copied
+from pinned host memory and its outputs copied back inside the timed region.
+``--impl reference`` times the float64 CPU oracle on the same workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+Under torchrun every rank runs an independent replica of the workload
+(the layer shards by video stream with no collective): weak scaling.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hybrid-attn layer tokens/s (21-frame 480p forward, 1 B200)"
+UNIT = "tokens/s"
+WORKLOAD_ID = 1
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    p.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def _cores():
+    return len(os.sched_getaffinity(0))
+
+
+def _config(w, extra=None):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "tokens_per_frame": w.T,
+         "frames": w.frames, "passes_per_frame": len(w.passes), "io_dtype": w.dtype,
+         "state_dtype": "fp32", "inputs": "all 21 frames resident in HBM (302 MB > 126 MB L2); "
+         "no L2 flush needed", "parallelism": "replicas (one independent stream per rank)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def oracle_frames(w, max_seconds, max_frames=None):
+    """Time the float64 oracle on consecutive frames of workload w (state carried)
+    until max_seconds of work or max_frames; returns (frames, seconds)."""
+    import torch
+    import oracle
+    import workloads as W
+    phi = [p.to(torch.float64).numpy() for p in W.feature_maps(w)]
+    S = W.zero_state(w)
+    done, spent = 0, 0.0
+    limit = max_frames or w.frames
+    while done < limit and spent < max_seconds:
+        q, k, v, g, bl = W.pass_inputs(w, done, 0).as_f64()
+        t0 = time.perf_counter()
+        for p, clean in enumerate(w.passes):
+            _, _, _, S = oracle.layer_pass(q, k, v, *phi, g, bl, S, clean)
+        spent += time.perf_counter() - t0
+        done += 1
+    return done, spent
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import workloads as W
+    w = W.WORKLOADS[WORKLOAD_ID]
+    # one step = one frame of the workload (all heads, one clean pass), oracle as it stands
+    oracle_frames(w, 1e9, max_frames=args.warmup)
+    times = []
+    for _ in range(args.steps):
+        n, s = oracle_frames(w, 1e9, max_frames=1)
+        times.append(s)
+    total = sum(times)
+    value = w.B * w.T * args.steps / total
+    sample = f"{args.steps} frames (1 step = 1 frame, all {w.H} heads, float64 NumPy oracle)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, {"step": "one frame"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover
+            self.nv, self.err = None, str(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    _NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+              0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+              0x100: "display_clock_setting"}
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self._NAMES.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                self._sample()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CUDA arm
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def attention_flops(w):
+    """Algorithmic FLOPs of one launch of the intra-frame attention kernel:
+    per (b, h) 4 T^2 d for softmax(QK^T)V plus 2 T d^2 for the inter-frame read
+    Q (phi_q^T S)."""
+    return w.B * w.H * (4.0 * w.T * w.T * w.d + 2.0 * w.T * w.d * w.d)
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+    import gated_delta_linear_b200 as G
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = W.WORKLOADS[WORKLOAD_ID]
+    phi = W.feature_maps(w)
+    layer = G.HybridAttention(w.B, w.H, w.T, w.d, w.torch_dtype, *phi, device=dev)
+    host = [W.pass_inputs(w, n, 0) for n in range(w.frames)]
+    frames = [[t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)] for x in host]
+    outs = [torch.empty_like(f[0]) for f in frames]
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    wsb = layer.workspace.numel()
+    phis = [p.data_ptr() for p in layer.phi]
+    state_ptr, ws_ptr = layer.state.data_ptr(), layer.workspace.data_ptr()
+    calls = [[f[0].data_ptr(), f[1].data_ptr(), f[2].data_ptr(), *phis, f[3].data_ptr(),
+              f[4].data_ptr(), state_ptr, 1, o.data_ptr(), ws_ptr, wsb, sptr]
+             for f, o in zip(frames, outs)]
+    desc = layer.desc
+    fwd = G.lib.hyb_attn_forward
+    import ctypes
+    dref = ctypes.byref(desc)
+
+    def step():
+        layer.state.zero_()
+        for c in calls:
+            st = fwd(dref, *c)
+            if st != G.HYB_OK:
+                raise G.HybAttnError(st, "hyb_attn_forward")
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch_cap = args.steps * w.frames * len(w.passes) * G.HYB_NUM_KERNELS + 16
+    assert G.hyb_attn_timing_begin(n_launch_cap) == G.HYB_OK
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    st, per_kernel, dropped = G.hyb_attn_timing_end()
+    assert st == G.HYB_OK and dropped == 0, (st, dropped)
+    ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = layer.device_status()
+
+    tokens_per_step = w.B * w.T * w.frames
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    launches = sum(v[0] for v in per_kernel.values())
+
+    # roofline of the dominant kernel, from its live event times
+    name = max(per_kernel, key=lambda k: per_kernel[k][1])
+    n_attn, ms_attn = per_kernel["intra_frame_attention"]
+    avg_attn_s = ms_attn / n_attn / 1e3
+    burst, sustained, hbm, src = _peaks()
+    achieved = attention_flops(w) / avg_attn_s / 1e12
+    roofline = {"kernel": "intra_frame_attention", "bound": "tensor", "achieved": achieved,
+                "peak": sustained, "unit": "TFLOP/s", "frac": achieved / sustained,
+                "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "traffic": None,
+                "avg_launch_us": avg_attn_s * 1e6,
+                "flops_per_launch": attention_flops(w),
+                "dominant_kernel_by_time": name,
+                "kernel_ms": {k: v[1] for k, v in per_kernel.items()},
+                "kernel_launches": {k: v[0] for k, v in per_kernel.items()}}
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tr = json.load(f)
+        if tr.get("kernel") == "intra_frame_attention" and tr.get("source_hash") == _src_hash():
+            roofline["traffic"] = tr["bytes_per_launch"]
+
+    # end to end through the C ABI with host buffers
+    e2e_steps = max(2, min(args.steps, 5))
+    pin = [[t.pin_memory() for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)] for x in host]
+    hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for f in pin for t in f)
+    d2h = sum(o.numel() * o.element_size() for o in hout)
+
+    def e2e_step():
+        layer.state.zero_()
+        for f, hf, c, o, ho in zip(frames, pin, calls, outs, hout):
+            for dst, src_ in zip(f, hf):
+                dst.copy_(src_, non_blocking=True)
+            st = fwd(dref, *c)
+            if st != G.HYB_OK:
+                raise G.HybAttnError(st, "hyb_attn_forward")
+            ho.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, s = oracle_frames(w, args.cpu_baseline_seconds)
+        cpu = {"value": w.B * w.T * n / s, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+               "sample": f"first {n} of {w.frames} frames (all {w.H} heads, state carried), "
+                         f"{s:.1f} s of float64 NumPy"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
+        "us_per_frame": 1e3 * ms / args.steps / w.frames,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded normals, video-DiT shapes)",
+        "config": _config(w),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "device_status": G.hyb_attn_status_string(status),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _src_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_linear_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,37 @@
+"""B200-native ARL2 hybrid attention layer.
+
+A thin ctypes binding of ``libhyb_attn.so`` (built from ``csrc/`` by
+``gated_delta_linear_b200.build``).  The functions carry the C names of
+``include/hyb_attn.h`` and only marshal arguments: every step of the layer
+runs in the library's CUDA kernels.  Importing this package fails loudly when
+the library has not been built.
+"""
+
+from ._binding import (  # noqa: F401
+    HYB_OK,
+    HYB_WARN_NONFINITE,
+    HYB_ERR_INVALID,
+    HYB_ERR_UNSUPPORTED,
+    HYB_ERR_ALIGN,
+    HYB_ERR_WORKSPACE,
+    HYB_ERR_CUDA,
+    HYB_ERR_TIMEOUT,
+    HYB_BF16,
+    HYB_FP32,
+    HybAttnDesc,
+    HybAttnError,
+    lib,
+    library_path,
+    make_desc,
+    hyb_attn_workspace_bytes,
+    hyb_attn_forward,
+    hyb_attn_forward_branches,
+    hyb_attn_get_device_status,
+    hyb_attn_status_string,
+    HybridAttention,
+    HybAttnTiming,
+    HYB_NUM_KERNELS,
+    hyb_attn_timing_begin,
+    hyb_attn_timing_end,
+    hyb_attn_kernel_name,
+)

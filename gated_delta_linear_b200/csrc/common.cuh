@@ -1,0 +1,66 @@
+// common.cuh -- shared device-side definitions of the hybrid attention library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hyb {
+
+// Device status flags, kept in the first word of the caller's workspace.
+enum : unsigned { FLAG_NONFINITE = 1u, FLAG_TIMEOUT = 2u };
+
+constexpr int kNumSMs = 148;          // B200
+constexpr int kUpdateTile = 128;      // tokens per key-tile of the state update
+constexpr size_t kStatusBytes = 256;  // status block at the start of the workspace
+
+// Everything one pass needs; built on the host from the C-ABI arguments.
+struct LayerArgs {
+    int B, H, T, D;
+    float sm_scale_log2;   // softmax scale * log2(e)
+    float l2_eps;
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* phi_q;
+    const void* phi_k;
+    const void* phi_v;
+    const float* gate_logits;
+    const float* beta_logits;
+    float* state;
+    void* out;
+    float* out_intra;
+    float* out_inter;
+    // workspace views
+    unsigned* flags;
+    float* W;                  // fp32 [BH][D][D]: phi_q^T S (SIMT path)
+    __nv_bfloat16* WT_hi;      // bf16 [BH][D][D]: (phi_q^T S)^T, high part (tensor path)
+    __nv_bfloat16* WT_lo;      // bf16 [BH][D][D]: low part
+    float* S_prev;             // fp32 [BH][D][D]: copy of S_{N-1} (clean pass)
+    float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
+    int nsplit;
+    int split_tokens;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+}  // namespace hyb

@@ -1,0 +1,313 @@
+// hyb_attn.cu -- C ABI of the ARL2 hybrid attention layer: argument checks,
+// workspace plan and the launch sequence of one pass.
+//
+// Source: "Technical summary: Attend Locally, Remember Linearly (ARL2)",
+// gist.science/ar/paper/2605.16579, §2.1 and §2.2; the interface contract is
+// documented in include/hyb_attn.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "hyb_attn.h"
+#include "common.cuh"
+#include "simt_layer.cuh"
+
+namespace {
+
+using namespace hyb;
+
+constexpr int kMaxDevices = 64;
+
+struct Plan {
+    int D;
+    bool bf16;
+    int nsplit;
+    int split_tokens;
+    size_t off_W, off_Sprev, off_part, total;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
+    if (!d) return HYB_ERR_INVALID;
+    if (d->B <= 0 || d->H <= 0 || d->T <= 0 || d->d_k <= 0 || d->d_v <= 0) return HYB_ERR_INVALID;
+    if (d->dtype != HYB_BF16 && d->dtype != HYB_FP32) return HYB_ERR_INVALID;
+    if (!(d->l2_eps >= 0.f) || !isfinite(d->l2_eps) || !isfinite(d->sm_scale)) return HYB_ERR_INVALID;
+    if (d->d_k != d->d_v) return HYB_ERR_UNSUPPORTED;
+    const int D = d->d_k;
+    const bool bf16 = d->dtype == HYB_BF16;
+    if (!((bf16 && D == 128) || (!bf16 && D == 32))) return HYB_ERR_UNSUPPORTED;
+    if (d->H > 65535 || d->B > 65535) return HYB_ERR_UNSUPPORTED;
+    const double elems = (double)d->B * d->T * d->H * D;
+    if (elems >= 2147483647.0) return HYB_ERR_UNSUPPORTED;
+    p->D = D;
+    p->bf16 = bf16;
+    // token splits of the state update: enough (b,h,split) blocks to cover the
+    // SMs, each split a whole number of 128-token tiles
+    const int BH = d->B * d->H;
+    const int ntiles = (d->T + kUpdateTile - 1) / kUpdateTile;
+    int want = (kNumSMs + BH - 1) / BH;
+    if (want > ntiles) want = ntiles;
+    if (want < 1) want = 1;
+    const int tiles_per_split = (ntiles + want - 1) / want;
+    p->split_tokens = tiles_per_split * kUpdateTile;
+    p->nsplit = (ntiles + tiles_per_split - 1) / tiles_per_split;
+    const size_t hh = (size_t)BH * D * D;
+    p->off_W = kStatusBytes;
+    p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
+    p->off_part = align_up(p->off_Sprev + hh * sizeof(float), 256);
+    p->total = align_up(p->off_part + hh * 2 * p->nsplit * sizeof(float), 256);
+    return HYB_OK;
+}
+
+// ---- optional kernel timing -------------------------------------------------
+enum { K_PREP = 0, K_ATTN = 1, K_PARTIALS = 2, K_APPLY = 3 };
+
+struct Timing {
+    bool on = false;
+    int cap = 0, used = 0, dropped = 0;
+    cudaEvent_t* ev = nullptr;   // 2 * cap events: start, stop per launch
+    int* kind = nullptr;
+} g_timing;
+
+// Launch through `fn`, bracketed by timing events when timing is on.
+template <typename F>
+cudaError_t timed(int kind, cudaStream_t st, F fn) {
+    if (!g_timing.on) {
+        fn();
+        return cudaSuccess;
+    }
+    if (g_timing.used >= g_timing.cap) {
+        ++g_timing.dropped;
+        fn();
+        return cudaSuccess;
+    }
+    const int i = g_timing.used++;
+    g_timing.kind[i] = kind;
+    cudaError_t e = cudaEventRecord(g_timing.ev[2 * i], st);
+    fn();
+    if (e == cudaSuccess) e = cudaEventRecord(g_timing.ev[2 * i + 1], st);
+    return e;
+}
+
+bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+// Opt each kernel into its dynamic shared memory once per device.
+template <typename K>
+cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done[dev] = 1;
+    return e;
+}
+
+template <int D, typename TIO>
+cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
+    static unsigned char done_attn[kMaxDevices], done_part[kMaxDevices], done_apply[kMaxDevices];
+    cudaError_t e;
+    const dim3 rows(D / 8, a.H, a.B);
+    const size_t attn_smem = simt::AttnSmem<D>::bytes;
+    const size_t ps = simt::PartialsSmem<D>::bytes;
+    const size_t as = simt::ApplySmem<D>::bytes;
+    if ((e = opt_in_smem(simt::attn_kernel<D, TIO>, attn_smem, done_attn)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(simt::partials_kernel<D, TIO>, ps, done_part)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(simt::apply_kernel<D, TIO>, as, done_apply)) != cudaSuccess) return e;
+    e = timed(K_PREP, st, [&] { simt::prep_kernel<D, TIO, false><<<rows, simt::kThreads, 0, st>>>(a, clean); });
+    if (e != cudaSuccess) return e;
+    const dim3 agrid((a.T + simt::AttnSmem<D>::BQ - 1) / simt::AttnSmem<D>::BQ, a.H, a.B);
+    e = timed(K_ATTN, st, [&] { simt::attn_kernel<D, TIO><<<agrid, simt::kThreads, attn_smem, st>>>(a); });
+    if (e != cudaSuccess) return e;
+    if (clean) {
+        e = timed(K_PARTIALS, st, [&] {
+            simt::partials_kernel<D, TIO><<<dim3(a.nsplit, a.H, a.B), simt::kThreads, ps, st>>>(a);
+        });
+        if (e != cudaSuccess) return e;
+        e = timed(K_APPLY, st, [&] { simt::apply_kernel<D, TIO><<<rows, simt::kThreads, as, st>>>(a); });
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
+hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                        const void* phi_q, const void* phi_k, const void* phi_v,
+                        const float* gate_logits, const float* beta_logits, float* state,
+                        int clean_pass, void* out, float* out_intra, float* out_inter,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    Plan p;
+    hyb_status s = make_plan(desc, &p);
+    if (s != HYB_OK) return s;
+    if (clean_pass != 0 && clean_pass != 1) return HYB_ERR_INVALID;
+    if (!q || !k || !v || !phi_q || !phi_k || !phi_v || !state) return HYB_ERR_INVALID;
+    if (!out && !(out_intra && out_inter)) return HYB_ERR_INVALID;
+    if ((out_intra == nullptr) != (out_inter == nullptr)) return HYB_ERR_INVALID;
+    if (clean_pass && (!gate_logits || !beta_logits)) return HYB_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, phi_q, phi_k, phi_v, state, out, out_intra, out_inter,
+                          gate_logits, beta_logits, workspace};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return HYB_ERR_ALIGN;
+    if (!workspace || workspace_bytes < p.total) return HYB_ERR_WORKSPACE;
+
+    LayerArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = desc->B;
+    a.H = desc->H;
+    a.T = desc->T;
+    a.D = p.D;
+    const float scale = desc->sm_scale > 0.f ? desc->sm_scale : 1.0f / sqrtf((float)desc->d_k);
+    a.sm_scale_log2 = scale * 1.4426950408889634f;
+    a.l2_eps = desc->l2_eps;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.phi_q = phi_q;
+    a.phi_k = phi_k;
+    a.phi_v = phi_v;
+    a.gate_logits = gate_logits;
+    a.beta_logits = beta_logits;
+    a.state = state;
+    a.out = out;
+    a.out_intra = out_intra;
+    a.out_inter = out_inter;
+    char* ws = (char*)workspace;
+    a.flags = (unsigned*)ws;
+    a.W = (float*)(ws + p.off_W);
+    a.WT_hi = (__nv_bfloat16*)(ws + p.off_W);
+    a.WT_lo = a.WT_hi + (size_t)a.B * a.H * p.D * p.D;
+    a.S_prev = (float*)(ws + p.off_Sprev);
+    a.partials = (float*)(ws + p.off_part);
+    a.nsplit = p.nsplit;
+    a.split_tokens = p.split_tokens;
+
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (p.bf16)
+        e = launch_simt<128, __nv_bfloat16>(a, clean_pass, st);
+    else
+        e = launch_simt<32, float>(a, clean_pass, st);
+    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyb_attn_workspace_bytes(const hyb_attn_desc* desc) {
+    Plan p;
+    return make_plan(desc, &p) == HYB_OK ? p.total : 0;
+}
+
+hyb_status hyb_attn_forward(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                            const void* phi_q, const void* phi_k, const void* phi_v,
+                            const float* gate_logits, const float* beta_logits, float* state,
+                            int clean_pass, void* out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    if (!out) return HYB_ERR_INVALID;
+    return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                        clean_pass, out, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc, const void* q, const void* k,
+                                     const void* v, const void* phi_q, const void* phi_k,
+                                     const void* phi_v, const float* gate_logits,
+                                     const float* beta_logits, float* state, int clean_pass,
+                                     void* out, float* out_intra, float* out_inter,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    if (!out_intra || !out_inter) return HYB_ERR_INVALID;
+    return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                        clean_pass, out, out_intra, out_inter, workspace, workspace_bytes, stream);
+}
+
+hyb_status hyb_attn_get_device_status(const void* workspace, void* stream) {
+    if (!workspace) return HYB_ERR_INVALID;
+    if (!aligned16(workspace)) return HYB_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HYB_ERR_CUDA;
+    unsigned flags = 0;
+    if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    if (flags && cudaMemset((void*)workspace, 0, sizeof(flags)) != cudaSuccess) return HYB_ERR_CUDA;
+    if (flags & FLAG_TIMEOUT) return HYB_ERR_TIMEOUT;
+    if (flags & FLAG_NONFINITE) return HYB_WARN_NONFINITE;
+    return HYB_OK;
+}
+
+hyb_status hyb_attn_timing_begin(int max_launches) {
+    if (g_timing.on || max_launches <= 0 || max_launches > (1 << 20)) return HYB_ERR_INVALID;
+    g_timing.ev = new (std::nothrow) cudaEvent_t[2 * (size_t)max_launches];
+    g_timing.kind = new (std::nothrow) int[max_launches];
+    if (!g_timing.ev || !g_timing.kind) {
+        delete[] g_timing.ev;
+        delete[] g_timing.kind;
+        g_timing.ev = nullptr;
+        g_timing.kind = nullptr;
+        return HYB_ERR_INVALID;
+    }
+    int made = 0;
+    for (; made < 2 * max_launches; ++made)
+        if (cudaEventCreate(&g_timing.ev[made]) != cudaSuccess) break;
+    if (made < 2 * max_launches) {
+        for (int i = 0; i < made; ++i) cudaEventDestroy(g_timing.ev[i]);
+        delete[] g_timing.ev;
+        delete[] g_timing.kind;
+        g_timing.ev = nullptr;
+        g_timing.kind = nullptr;
+        return HYB_ERR_CUDA;
+    }
+    g_timing.cap = max_launches;
+    g_timing.used = 0;
+    g_timing.dropped = 0;
+    g_timing.on = true;
+    return HYB_OK;
+}
+
+hyb_status hyb_attn_timing_end(hyb_attn_timing* out) {
+    if (!g_timing.on) return HYB_ERR_INVALID;
+    hyb_status st = HYB_OK;
+    hyb_attn_timing t;
+    memset(&t, 0, sizeof(t));
+    for (int i = 0; i < g_timing.used; ++i) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(g_timing.ev[2 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, g_timing.ev[2 * i], g_timing.ev[2 * i + 1]) != cudaSuccess) {
+            st = HYB_ERR_CUDA;
+            continue;
+        }
+        t.launches[g_timing.kind[i]] += 1;
+        t.total_ms[g_timing.kind[i]] += ms;
+    }
+    t.dropped = g_timing.dropped;
+    for (int i = 0; i < 2 * g_timing.cap; ++i) cudaEventDestroy(g_timing.ev[i]);
+    delete[] g_timing.ev;
+    delete[] g_timing.kind;
+    g_timing = Timing();
+    if (out) *out = t;
+    return st;
+}
+
+const char* hyb_attn_kernel_name(int kernel) {
+    static const char* names[HYB_NUM_KERNELS] = {"prep", "intra_frame_attention",
+                                                 "delta_update_partials", "delta_update_apply"};
+    return (kernel >= 0 && kernel < HYB_NUM_KERNELS) ? names[kernel] : nullptr;
+}
+
+const char* hyb_attn_status_string(hyb_status s) {
+    switch (s) {
+        case HYB_OK: return "HYB_OK";
+        case HYB_WARN_NONFINITE: return "HYB_WARN_NONFINITE: a state update produced inf/NaN";
+        case HYB_ERR_INVALID: return "HYB_ERR_INVALID: invalid argument";
+        case HYB_ERR_UNSUPPORTED: return "HYB_ERR_UNSUPPORTED: unsupported dtype/shape";
+        case HYB_ERR_ALIGN: return "HYB_ERR_ALIGN: pointer not 16-byte aligned";
+        case HYB_ERR_WORKSPACE: return "HYB_ERR_WORKSPACE: workspace missing or too small";
+        case HYB_ERR_CUDA: return "HYB_ERR_CUDA: CUDA call or launch failed";
+        case HYB_ERR_TIMEOUT: return "HYB_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown hyb_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+/*
+ * hyb_attn.h -- C ABI of the ARL2 hybrid attention layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Technical summary: Attend Locally, Remember Linearly (ARL2)",
+ * gist.science/ar/paper/2605.16579) splits the self-attention of an
+ * autoregressive video diffusion transformer into two branches:
+ *
+ *   §2.1 intra-frame branch   O_intra = softmax(Q K^T * sm_scale) V over the
+ *                             tokens of the current frame, bidirectional.
+ *   §2.1 inter-frame branch   O_inter = Q' S_{N-1}, with Q' = Q phi_q^T and a
+ *                             fixed-size per-head fp32 state S (d_k x d_v).
+ *   §2.1 state update         S_N = alpha S_{N-1} + K'^T diag(beta) (V' - K' S_{N-1})
+ *                             (printed garbled on the page; this is the only
+ *                             shape-consistent reading), K' = rownorm(K phi_k^T),
+ *                             V' = V phi_v^T, beta_t = sigmoid(beta_logit_t),
+ *                             alpha = mean_t sigmoid(gate_logit_t) (one forget
+ *                             gate per head and frame, §4 "headwise gating").
+ *   §2.2 frame-level access   every token of a frame reads the same pre-update
+ *                             S_{N-1}; the state is written after the reads.
+ *   §2.2 clean-pass updates   denoising passes (clean_pass = 0) read S and never
+ *                             write it; the final clean pass (clean_pass = 1)
+ *                             writes it once.
+ *
+ * Readings where the pages are silent (all are choices of this library):
+ *   - output      out = O_intra + O_inter, rounded once to the I/O dtype
+ *                 (the pages do not say how the branches combine);
+ *   - 1x1 maps    x'[o] = sum_i phi[o][i] x[i], i.e. X' = X phi^T; no bias,
+ *                 no nonlinearity; the same q, k, v feed both branches;
+ *   - K' only     is L2-normalised, as k / sqrt(sum k^2 + l2_eps);
+ *   - sm_scale    defaults to 1/sqrt(d_k);
+ *   - alpha       is the mean of the per-token sigmoids, not the sigmoid of
+ *                 the mean logit.
+ *
+ * Layouts (row-major, contiguous, every pointer 16-byte aligned):
+ *   q, k, v, out          [B][T][H][d]     dtype (bf16 or fp32)
+ *   phi_q, phi_k, phi_v   [H][d][d]        dtype, phi[h][o][i]
+ *   gate_logits,
+ *   beta_logits           [B][H][T]        fp32 (read only when clean_pass)
+ *   state                 [B][H][d_k][d_v] fp32, read always, written only
+ *                                           when clean_pass
+ *   out_intra, out_inter  [B][T][H][d]     fp32 (debug entry point)
+ *
+ * Supported shapes: d_k == d_v == 128 with bf16 I/O (tensor-core path), and
+ * d_k == d_v == 32 with fp32 I/O (fp32 SIMT path).  Any T >= 1, B >= 1, H >= 1
+ * with B*H*T*d below 2^31 elements.  Other combinations return
+ * HYB_ERR_UNSUPPORTED.
+ *
+ * Ownership: the caller owns every buffer, including the persistent state and
+ * the workspace; the library never allocates, frees or synchronises inside
+ * hyb_attn_forward*.  The state persists across calls: the caller passes
+ * S_{N-1} for frame N and zero-fills it for S_0.  The caller zero-fills the
+ * workspace once after allocating it (its first 256 bytes hold the device
+ * status flags).  Calls are asynchronous on the given stream; argument errors
+ * are reported before anything is launched.  `stream` is a cudaStream_t
+ * (NULL = legacy default stream).  Calls sharing one workspace must be ordered
+ * on one stream.  No C++ exception crosses this interface.
+ */
+#ifndef HYB_ATTN_H
+#define HYB_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HYB_OK = 0,
+    HYB_WARN_NONFINITE = 1,   /* device flag: a state update produced inf/NaN      */
+    HYB_ERR_INVALID = -1,     /* null pointer, non-positive size, bad flag          */
+    HYB_ERR_UNSUPPORTED = -2, /* (dtype, d) combination not built                   */
+    HYB_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned                   */
+    HYB_ERR_WORKSPACE = -4,   /* workspace null or smaller than hyb_attn_workspace_bytes */
+    HYB_ERR_CUDA = -5,        /* a CUDA runtime/driver call or a launch failed      */
+    HYB_ERR_TIMEOUT = -6      /* device flag: a bounded device-side wait gave up    */
+} hyb_status;
+
+typedef enum { HYB_BF16 = 0, HYB_FP32 = 1 } hyb_dtype;
+
+typedef struct {
+    int B, H, T, d_k, d_v;
+    int dtype;        /* hyb_dtype: dtype of q, k, v, phi_*, out                 */
+    float sm_scale;   /* softmax scale; <= 0 selects 1/sqrt(d_k)                 */
+    float l2_eps;     /* key-normalisation epsilon (>= 0); 1e-6 is the default   */
+} hyb_attn_desc;
+
+/* Bytes of device workspace one call with this descriptor needs (0 if the
+ * descriptor is invalid or unsupported).  It is linear in B*H and does not
+ * depend on the frame count. */
+size_t hyb_attn_workspace_bytes(const hyb_attn_desc* desc);
+
+/* One pass of the layer over one frame (ARL2 summary §2.1, §2.2).
+ * clean_pass = 0: query-only denoising pass; reads state, never writes it;
+ *                 gate_logits / beta_logits may be NULL.
+ * clean_pass = 1: also applies the gated delta update to state in place,
+ *                 after every read of S_{N-1} for this frame's output.
+ * Writes out = O_intra + O_inter.  Returns HYB_OK once the work is enqueued. */
+hyb_status hyb_attn_forward(const hyb_attn_desc* desc,
+                            const void* q, const void* k, const void* v,
+                            const void* phi_q, const void* phi_k, const void* phi_v,
+                            const float* gate_logits, const float* beta_logits,
+                            float* state, int clean_pass, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Same pass, also writing the two branches separately in fp32 (for parity
+ * checks); out may be NULL, out_intra and out_inter may not. */
+hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
+                                     const void* q, const void* k, const void* v,
+                                     const void* phi_q, const void* phi_k, const void* phi_v,
+                                     const float* gate_logits, const float* beta_logits,
+                                     float* state, int clean_pass, void* out,
+                                     float* out_intra, float* out_inter,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status flags kept
+ * in `workspace`: HYB_ERR_TIMEOUT if a bounded device wait gave up,
+ * else HYB_WARN_NONFINITE if a state update produced inf/NaN since the last
+ * read, else HYB_OK (or HYB_ERR_CUDA if the synchronisation failed). */
+hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
+
+/* ---- optional kernel timing (benchmarks) ------------------------------------
+ * Process-wide and off by default.  hyb_attn_timing_begin(n) creates 2n CUDA
+ * events on the current device; until hyb_attn_timing_end, every kernel that
+ * hyb_attn_forward* launches is bracketed by two of them on the call's stream
+ * (launches beyond n are counted as dropped).  Do not leave timing on while a
+ * stream is being captured into a CUDA graph.  hyb_attn_timing_end waits for
+ * the recorded events, sums each kernel's launch count and event time into
+ * *out, destroys the events and turns timing off.  Not thread-safe. */
+#define HYB_NUM_KERNELS 4
+typedef struct {
+    int launches[HYB_NUM_KERNELS];     /* indexed as hyb_attn_kernel_name() */
+    double total_ms[HYB_NUM_KERNELS];
+    int dropped;
+} hyb_attn_timing;
+
+hyb_status hyb_attn_timing_begin(int max_launches);
+hyb_status hyb_attn_timing_end(hyb_attn_timing* out);
+/* "prep", "intra_frame_attention", "delta_update_partials", "delta_update_apply"; NULL if out of range */
+const char* hyb_attn_kernel_name(int kernel);
+
+/* Static string naming a status code. */
+const char* hyb_attn_status_string(hyb_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYB_ATTN_H */

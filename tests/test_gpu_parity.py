@@ -1,0 +1,202 @@
+"""Parity of the CUDA library (through its C ABI) against the float64 oracle.
+
+All five workloads run at their full sizes on the GPU; where the oracle would
+take minutes, it checks sampled (batch, head) pairs of every pass.  Bounds and
+their derivation: tests/tolerances.py.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from tests import tolerances as tol
+from tests.harness import Run, f64, oracle_state_from_prior_frames, phis
+
+pytestmark = pytest.mark.gpu
+
+
+def _frames(run, frames, passes, check=True):
+    for n in range(frames):
+        for p, clean in enumerate(passes):
+            run.step(n, p, clean, check=check)
+        if any(passes):
+            bound = tol.STATE_BF16 if run.w.dtype == "bf16" else tol.STATE_FP32
+            assert run.worst["state"] <= bound, f"state after frame {n}: {run.worst['state']:.3e}"
+
+
+def test_tiny_fp32_workload_all_passes():
+    w = W.WORKLOADS[0]
+    run = Run(w)
+    _frames(run, w.frames, w.passes)
+    assert run.worst["state"] <= tol.STATE_FP32
+    print("worst", run.worst)
+
+
+def test_wan_480p_21_frames():
+    w = W.WORKLOADS[1]
+    run = Run(w)
+    _frames(run, w.frames, w.passes)
+    assert run.state_error() <= tol.STATE_BF16
+    print("worst", run.worst)
+
+
+def test_wan14b_streaming_step_on_prebuilt_state():
+    w = W.WORKLOADS[2]
+    phi64 = [f64(p) for p in phis(w)]
+    S0 = oracle_state_from_prior_frames(w, phi64).astype(np.float32).astype(np.float64)
+    heads = [(0, h) for h in (0, 7, 19, 31, 39)]
+    run = Run(w, heads=heads, state0=S0)
+    _frames(run, w.frames, w.passes)
+    print("worst", run.worst)
+
+
+@pytest.mark.slow
+def test_720p_21_frames_sampled_heads():
+    w = W.WORKLOADS[3]
+    run = Run(w, heads=[(0, 0), (0, 21), (0, 39)])
+    _frames(run, w.frames, w.passes)
+    assert run.state_error() <= tol.STATE_BF16
+    print("worst", run.worst)
+
+
+
+
+def test_long_stream_constant_memory_and_parity():
+    w = W.WORKLOADS[4]
+    heads = [(0, 3), (1, 10)]
+    run = Run(w, heads=heads, check_branches=False)
+    G = run.G
+    fmax = float(np.finfo(np.float32).max)
+    mem = {}
+    checked = 0
+    overflowed = False
+    for n in range(w.frames):
+        check = not overflowed
+        run.step(n, 0, True, check=check)
+        if check:
+            big = max(np.abs(run.S_ref[b, h]).max() for b, h in heads)
+            if big > fmax / 1e4:       # the oracle's state is about to leave the fp32 range
+                overflowed = True
+            else:
+                checked = n + 1
+                assert run.worst["state"] <= tol.STATE_BF16, (n, run.worst)
+        if n + 1 in (1, 60, 120, 240):
+            torch.cuda.synchronize()
+            mem[n + 1] = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+    assert checked >= 50, checked
+    allocs = {v[0] for v in mem.values()}
+    frees = {v[1] for v in mem.values()}
+    assert len(allocs) == 1 and len(frees) == 1, mem
+    st = run.layer.device_status()
+    if overflowed:
+        assert st == G.HYB_WARN_NONFINITE, G.hyb_attn_status_string(st)
+    assert run.layer.device_status() == G.HYB_OK   # flags clear after reading
+    print("checked frames", checked, "worst", run.worst)
+
+
+@pytest.mark.parametrize("T", [1, 17, 127, 128, 129, 300])
+def test_ragged_frame_lengths_bf16(T):
+    base = W.WORKLOADS[1]
+    w = W.small_workload(base, H=3, T=T, frames=3, passes=(False, True))
+    run = Run(w)
+    _frames(run, w.frames, w.passes)
+    print(T, "worst", run.worst)
+
+
+@pytest.mark.parametrize("T", [1, 33, 200])
+def test_ragged_frame_lengths_fp32(T):
+    w = W.small_workload(W.WORKLOADS[0], T=T, frames=3)
+    run = Run(w)
+    _frames(run, w.frames, w.passes)
+
+
+def _layer(w):
+    import gated_delta_linear_b200 as G
+    return G.HybridAttention(w.B, w.H, w.T, w.d, w.torch_dtype, *phis(w))
+
+
+def _dev_inputs(w, n, p):
+    inp = W.pass_inputs(w, n, p)
+    return [t.cuda() for t in (inp.q, inp.k, inp.v, inp.gate_logits, inp.beta_logits)]
+
+
+def test_query_only_pass_leaves_state_bit_identical():
+    w = W.small_workload(W.WORKLOADS[1], frames=2)
+    L = _layer(w)
+    q, k, v, g, bl = _dev_inputs(w, 0, 0)
+    L.forward(q, k, v, g, bl, True)
+    before = L.state.clone()
+    for p in range(3):
+        q, k, v, g, bl = _dev_inputs(w, 1, p)
+        L.forward(q, k, v, g, bl, False)
+        L.forward(q, k, v, None, None, False)
+    torch.cuda.synchronize()
+    assert torch.equal(before, L.state)
+
+
+def test_forward_equals_branches_and_is_deterministic():
+    w = W.small_workload(W.WORKLOADS[1], frames=3)
+    outs = []
+    for mode in ("forward", "branches", "forward"):
+        L = _layer(w)
+        o = None
+        for n in range(w.frames):
+            q, k, v, g, bl = _dev_inputs(w, n, 0)
+            if mode == "forward":
+                o = L.forward(q, k, v, g, bl, True)
+            else:
+                o, oi, oe = L.forward_branches(q, k, v, g, bl, True)
+        torch.cuda.synchronize()
+        outs.append((o.clone(), L.state.clone()))
+    for o, s in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
+
+
+def test_checkpoint_resume_bit_identical():
+    w = W.WORKLOADS[1]
+
+    def run(frames_a, frames_b):
+        L = _layer(w)
+        outs = []
+        for n in range(frames_a):
+            outs.append(L.forward(*_dev_inputs(w, n, 0), True).clone())
+        saved = L.state.cpu().clone()
+        L2 = _layer(w)
+        L2.state.copy_(saved.cuda())
+        for n in range(frames_a, frames_a + frames_b):
+            outs.append(L2.forward(*_dev_inputs(w, n, 0), True).clone())
+        torch.cuda.synchronize()
+        return outs, L2.state.clone()
+
+    o1, s1 = run(21, 0)
+    o2, s2 = run(10, 11)
+    assert torch.equal(s1, s2)
+    for a, b in zip(o1, o2):
+        assert torch.equal(a, b)
+
+
+def test_nonfinite_state_is_reported():
+    import gated_delta_linear_b200 as G
+    w = W.small_workload(W.WORKLOADS[1], H=2, T=256, frames=1)
+    L = _layer(w)
+    assert L.device_status() == G.HYB_OK
+    L.state.fill_(3e38)
+    L.forward(*_dev_inputs(w, 0, 0), True)
+    assert L.device_status() == G.HYB_WARN_NONFINITE
+    assert L.device_status() == G.HYB_OK
+
+
+def test_device_side_argument_errors():
+    import gated_delta_linear_b200 as G
+    w = W.small_workload(W.WORKLOADS[1], H=2, T=64, frames=1)
+    L = _layer(w)
+    q, k, v, g, bl = _dev_inputs(w, 0, 0)
+    out = torch.empty_like(q)
+    small = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    st = G.hyb_attn_forward(L.desc, q, k, v, *L.phi, g, bl, L.state, 1, out, small)
+    assert st == G.HYB_ERR_WORKSPACE
+    qq = torch.empty(q.numel() + 8, dtype=q.dtype, device="cuda")
+    st = G.hyb_attn_forward(L.desc, qq.data_ptr() + 2, k, v, *L.phi, g, bl, L.state, 1, out,
+                            L.workspace)
+    assert st == G.HYB_ERR_ALIGN
