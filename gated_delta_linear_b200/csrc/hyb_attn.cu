@@ -13,6 +13,7 @@
 #include "hyb_attn.h"
 #include "common.cuh"
 #include "simt_layer.cuh"
+#include "tc_kernels.cuh"
 
 namespace {
 
@@ -134,6 +135,80 @@ cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// ---- tensor-core path (bf16, d = 128) ----------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor map with 64 x 128 x 1 boxes and 128-byte swizzle:
+// dims {d0 (contiguous), d1, d2}, byte strides s1, s2 of dims 1 and 2.
+bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+           uint64_t s2) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1, s2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
+    using bf16 = __nv_bfloat16;
+    static unsigned char done_attn[kMaxDevices], done_part[kMaxDevices], done_apply[kMaxDevices];
+    constexpr int D = 128;
+    cudaError_t e;
+    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::partials_kernel, tc::upd::SMEM, done_part)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(simt::apply_kernel<D, bf16>, simt::ApplySmem<D>::bytes, done_apply)) != cudaSuccess)
+        return e;
+    const uint64_t row_bytes = (uint64_t)a.H * D * 2;
+    const uint64_t bh = (uint64_t)a.B * a.H;
+    CUtensorMap tq, tk, tv, tw, tphik;
+    if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+        !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+        !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+        !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
+        !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2))
+        return cudaErrorInvalidValue;
+    const dim3 rows(D / 8, a.H, a.B);
+    e = timed(K_PREP, st, [&] { simt::prep_kernel<D, bf16, true><<<rows, simt::kThreads, 0, st>>>(a, clean); });
+    if (e != cudaSuccess) return e;
+    const dim3 agrid((a.T + tc::kTile - 1) / tc::kTile, a.H, a.B);
+    e = timed(K_ATTN, st, [&] {
+        tc::attention_kernel<<<agrid, tc::attn::kThreads, tc::attn::SMEM, st>>>(a, tq, tk, tv, tw);
+    });
+    if (e != cudaSuccess) return e;
+    if (clean) {
+        e = timed(K_PARTIALS, st, [&] {
+            tc::partials_kernel<<<dim3(a.nsplit, a.H, a.B), tc::upd::kThreads, tc::upd::SMEM, st>>>(a, tk, tv,
+                                                                                                  tphik);
+        });
+        if (e != cudaSuccess) return e;
+        e = timed(K_APPLY, st, [&] {
+            simt::apply_kernel<D, bf16><<<rows, simt::kThreads, simt::ApplySmem<D>::bytes, st>>>(a);
+        });
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
 hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
                         const void* phi_q, const void* phi_k, const void* phi_v,
                         const float* gate_logits, const float* beta_logits, float* state,
@@ -187,7 +262,7 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     if (p.bf16)
-        e = launch_simt<128, __nv_bfloat16>(a, clean_pass, st);
+        e = launch_tc(a, clean_pass, st);
     else
         e = launch_simt<32, float>(a, clean_pass, st);
     return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
