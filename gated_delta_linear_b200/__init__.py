@@ -1,7 +1,7 @@
 """B200-native ARL2 hybrid attention layer.
 
 A thin ctypes binding of ``libhyb_attn.so`` (built from ``csrc/`` by
-``gated_delta_linear_b200.build``).  The functions carry the C names of
+``gated_delta_linear_b200/build.py``).  The functions carry the C names of
 ``include/hyb_attn.h`` and only marshal arguments: every step of the layer
 runs in the library's CUDA kernels.  Importing this package fails loudly when
 the library has not been built.

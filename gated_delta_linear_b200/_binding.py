@@ -47,7 +47,7 @@ class HybAttnTiming(ctypes.Structure):
 def _load():
     if not os.path.exists(library_path):
         raise ImportError(
-            f"{library_path} is missing: build it with `python -m gated_delta_linear_b200.build`")
+            f"{library_path} is missing: build it with `python gated_delta_linear_b200/build.py`")
     L = ctypes.CDLL(library_path)
     vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     dp = ctypes.POINTER(HybAttnDesc)

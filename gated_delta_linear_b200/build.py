@@ -1,6 +1,7 @@
 """Build libhyb_attn.so in-tree with nvcc for sm_100a (B200).
 
-Usage: ``python -m gated_delta_linear_b200.build`` (or ``build()`` from Python).
+Usage: ``python gated_delta_linear_b200/build.py [--force] [-v]`` (run as a script:
+importing the package needs the library already built).
 """
 
 from __future__ import annotations
