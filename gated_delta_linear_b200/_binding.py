@@ -58,6 +58,8 @@ def _load():
     L.hyb_attn_forward_branches.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp,
                                             vp, vp, vp, sz, vp]
     L.hyb_attn_forward_branches.restype = i
+    L.hyb_attn_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
+    L.hyb_attn_forward_noalloc.restype = i
     L.hyb_attn_get_device_status.argtypes = [vp, vp]
     L.hyb_attn_get_device_status.restype = i
     L.hyb_attn_timing_begin.argtypes = [i]
@@ -119,6 +121,19 @@ def hyb_attn_forward_branches(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, b
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(phi_q), _ptr(phi_k), _ptr(phi_v),
         _ptr(gate_logits), _ptr(beta_logits), _ptr(state), int(clean_pass), _ptr(out),
         _ptr(out_intra), _ptr(out_inter), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+HYB_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                             clean_pass, out, stream=None) -> int:
+    """hyb_attn_forward without a workspace argument, for callers that cannot
+    allocate device memory; uses the library's fixed scratch array instead."""
+    return lib.hyb_attn_forward_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(phi_q), _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits),
+                                        _ptr(beta_logits), _ptr(state), int(clean_pass), _ptr(out),
+                                        _stream(stream))
 
 
 def hyb_attn_get_device_status(workspace, stream=None) -> int:

@@ -386,3 +386,53 @@ const char* hyb_attn_status_string(hyb_status s) {
 }
 
 }  // extern "C"
+
+// ---- zero-allocation variant --------------------------------------------------
+// Scratch for hyb_attn_forward_noalloc: a fixed array in the library's own
+// device memory, so that callers which may not allocate (graph capture in a
+// strict mode, allocator callbacks, fixed-budget serving loops) can run a pass
+// without a workspace.  Every GPU that loads the library holds it until exit.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HYB_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_noalloc_scratch per device, looked up once with that
+// device current.  In host code the array's name is only a host-side stand-in.
+void* g_noalloc_ptr[kMaxDevices];
+
+void* noalloc_scratch(cudaError_t* err) {
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        *err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc, const void* q, const void* k,
+                                               const void* v, const void* phi_q, const void* phi_k,
+                                               const void* phi_v, const float* gate_logits,
+                                               const float* beta_logits, float* state, int clean_pass,
+                                               void* out, void* stream) {
+    if (!out) return HYB_ERR_INVALID;
+    Plan p;
+    hyb_status s = make_plan(desc, &p);
+    if (s != HYB_OK) return s;
+    if (p.total > (size_t)HYB_NOALLOC_SCRATCH_BYTES) return HYB_ERR_WORKSPACE;
+    cudaError_t e;
+    void* scratch = noalloc_scratch(&e);
+    if (!scratch) return HYB_ERR_CUDA;
+    // the status word accumulates flags: start every call from zero
+    if (cudaMemsetAsync(scratch, 0, sizeof(unsigned), (cudaStream_t)stream) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                        clean_pass, out, nullptr, nullptr, scratch, HYB_NOALLOC_SCRATCH_BYTES, stream);
+}

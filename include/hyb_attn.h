@@ -112,6 +112,33 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
                                      float* out_intra, float* out_inter,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* hyb_attn_forward_noalloc -- the same pass as hyb_attn_forward for callers
+ * that cannot allocate device memory: code running where cudaMalloc is
+ * forbidden or unavailable (inside a CUDA graph being captured with a strict
+ * capture mode, inside an allocator or memory-pool callback, in a real-time
+ * or pre-sized serving loop whose memory budget is fixed up front).  No
+ * counterpart in the paper: this is an interface convenience only.
+ *
+ * Instead of a caller workspace it uses one scratch array of
+ * HYB_NOALLOC_SCRATCH_BYTES held by the library on every GPU that loads it,
+ * for as long as the process runs.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine); the caller still passes every input
+ * and output.  A descriptor whose hyb_attn_workspace_bytes() exceeds
+ * HYB_NOALLOC_SCRATCH_BYTES is rejected with HYB_ERR_WORKSPACE before any
+ * launch.  The first call on a device looks up the scratch array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls on a device share the one array
+ * and it keeps the last call's contents: calls that can overlap on the GPU
+ * (different streams, concurrent threads) race on it and must be serialised by
+ * the caller.  Device status flags of these calls are cleared at the start of
+ * each call and are not reported by hyb_attn_get_device_status. */
+#define HYB_NOALLOC_SCRATCH_BYTES (32u << 20)
+hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc,
+                                    const void* q, const void* k, const void* v,
+                                    const void* phi_q, const void* phi_k, const void* phi_v,
+                                    const float* gate_logits, const float* beta_logits,
+                                    float* state, int clean_pass, void* out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status flags kept
  * in `workspace`: HYB_ERR_TIMEOUT if a bounded device wait gave up,
  * else HYB_WARN_NONFINITE if a state update produced inf/NaN since the last
