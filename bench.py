@@ -47,6 +47,9 @@ def _args():
     p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     p.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-run", action="store_true",
+                   help="3 warm-up frames then one frame of the 480p workload; no JSON line "
+                        "(a small, fixed launch sequence for ncu captures)")
     return p.parse_args()
 
 
@@ -235,6 +238,14 @@ def run_cuda(args):
             st = fwd(dref, *c)
             if st != G.HYB_OK:
                 raise G.HybAttnError(st, "hyb_attn_forward")
+
+    if args.profile_run:
+        # kernel order per frame: prep, intra_frame_attention, delta_update_partials, delta_update_apply
+        for c in calls[:4]:
+            assert fwd(dref, *c) == G.HYB_OK
+        torch.cuda.synchronize(dev)
+        print("profile run done: 4 frames x 4 kernels", flush=True)
+        return 0
 
     for _ in range(max(3, args.warmup)):
         step()

@@ -110,16 +110,21 @@ cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
 
 template <int D, typename TIO>
 cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
-    static unsigned char done_attn[kMaxDevices], done_part[kMaxDevices], done_apply[kMaxDevices];
+    static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_part[kMaxDevices],
+        done_apply[kMaxDevices];
     cudaError_t e;
-    const dim3 rows(D / 8, a.H, a.B);
+    const dim3 rows(D / simt::kRows, a.H, a.B);
+    const size_t prep_smem = simt::PrepSmem<D>::bytes;
     const size_t attn_smem = simt::AttnSmem<D>::bytes;
     const size_t ps = simt::PartialsSmem<D>::bytes;
-    const size_t as = simt::ApplySmem<D>::bytes;
+    const size_t as = simt::ApplySmem<D, TIO>::bytes;
+    if ((e = opt_in_smem(simt::prep_kernel<D, TIO, false>, prep_smem, done_prep)) != cudaSuccess) return e;
     if ((e = opt_in_smem(simt::attn_kernel<D, TIO>, attn_smem, done_attn)) != cudaSuccess) return e;
     if ((e = opt_in_smem(simt::partials_kernel<D, TIO>, ps, done_part)) != cudaSuccess) return e;
     if ((e = opt_in_smem(simt::apply_kernel<D, TIO>, as, done_apply)) != cudaSuccess) return e;
-    e = timed(K_PREP, st, [&] { simt::prep_kernel<D, TIO, false><<<rows, simt::kThreads, 0, st>>>(a, clean); });
+    e = timed(K_PREP, st, [&] {
+        simt::prep_kernel<D, TIO, false><<<rows, simt::kThreads, prep_smem, st>>>(a, clean);
+    });
     if (e != cudaSuccess) return e;
     const dim3 agrid((a.T + simt::AttnSmem<D>::BQ - 1) / simt::AttnSmem<D>::BQ, a.H, a.B);
     e = timed(K_ATTN, st, [&] { simt::attn_kernel<D, TIO><<<agrid, simt::kThreads, attn_smem, st>>>(a); });
@@ -171,13 +176,16 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
 
 cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     using bf16 = __nv_bfloat16;
-    static unsigned char done_attn[kMaxDevices], done_part[kMaxDevices], done_apply[kMaxDevices];
+    static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_part[kMaxDevices],
+        done_apply[kMaxDevices];
     constexpr int D = 128;
     cudaError_t e;
     if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
     if ((e = opt_in_smem(tc::partials_kernel, tc::upd::SMEM, done_part)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(simt::apply_kernel<D, bf16>, simt::ApplySmem<D>::bytes, done_apply)) != cudaSuccess)
-        return e;
+    const size_t prep_smem = simt::PrepSmem<D>::bytes;
+    const size_t apply_smem = simt::ApplySmem<D, bf16>::bytes;
+    if ((e = opt_in_smem(simt::prep_kernel<D, bf16, true>, prep_smem, done_prep)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(simt::apply_kernel<D, bf16>, apply_smem, done_apply)) != cudaSuccess) return e;
     const uint64_t row_bytes = (uint64_t)a.H * D * 2;
     const uint64_t bh = (uint64_t)a.B * a.H;
     CUtensorMap tq, tk, tv, tw, tphik;
@@ -187,8 +195,10 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
         !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
         !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2))
         return cudaErrorInvalidValue;
-    const dim3 rows(D / 8, a.H, a.B);
-    e = timed(K_PREP, st, [&] { simt::prep_kernel<D, bf16, true><<<rows, simt::kThreads, 0, st>>>(a, clean); });
+    const dim3 rows(D / simt::kRows, a.H, a.B);
+    e = timed(K_PREP, st, [&] {
+        simt::prep_kernel<D, bf16, true><<<rows, simt::kThreads, prep_smem, st>>>(a, clean);
+    });
     if (e != cudaSuccess) return e;
     const dim3 agrid((a.T + tc::kTile - 1) / tc::kTile, a.H, a.B);
     e = timed(K_ATTN, st, [&] {
@@ -202,7 +212,7 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
         });
         if (e != cudaSuccess) return e;
         e = timed(K_APPLY, st, [&] {
-            simt::apply_kernel<D, bf16><<<rows, simt::kThreads, simt::ApplySmem<D>::bytes, st>>>(a);
+            simt::apply_kernel<D, bf16><<<rows, simt::kThreads, apply_smem, st>>>(a);
         });
         if (e != cudaSuccess) return e;
     }

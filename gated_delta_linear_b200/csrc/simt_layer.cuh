@@ -26,36 +26,79 @@ namespace simt {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- prep
-// grid (D/8, H, B); warp w of block x handles row k = 8x + w of W.
+// grid (D/16, H, B): block x computes rows k0..k0+15 of W = phi_q^T S.  S and the
+// block's 16 columns of phi_q are staged in shared memory; each warp owns two
+// rows of W and every lane the columns lane + 32c.
+constexpr int kRows = 16;
+
+template <int D>
+struct PrepSmem {
+    static constexpr size_t bytes = sizeof(float) * (D * D + D * kRows + kRows * (D + 1));
+};
+
 template <int D, typename TIO, bool kSplitOut>
 __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) {
     constexpr int NC = D / 32;
-    const int b = blockIdx.z, h = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kk = blockIdx.x * 8 + warp;
+    extern __shared__ float smem[];
+    float* Ss = smem;                  // [D][D]     S_{N-1}
+    float* Ph = Ss + D * D;            // [D][16]    phi_q[o][k0 + kr]
+    float* Wst = Ph + D * kRows;       // [16][D+1]  W rows (for the transposed split store)
+    const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * kRows;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
-    const float* S = a.state + bh * D * D;
+    const float4* S4 = reinterpret_cast<const float4*>(a.state + bh * D * D);
+    for (int i = tid; i < D * D / 4; i += kThreads) reinterpret_cast<float4*>(Ss)[i] = S4[i];
     const TIO* phiq = (const TIO*)a.phi_q + (size_t)h * D * D;
-    float acc[NC];
+    for (int i = tid; i < D * kRows; i += kThreads) Ph[i] = to_f32(phiq[(i / kRows) * D + k0 + i % kRows]);
+    __syncthreads();
+    const int r0 = 2 * warp;
+    float acc[2][NC];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) acc[c] = 0.f;
+    for (int c = 0; c < NC; ++c) acc[0][c] = acc[1][c] = 0.f;
+#pragma unroll 4
     for (int o = 0; o < D; ++o) {
-        const float p = to_f32(phiq[o * D + kk]);
+        const float p0 = Ph[o * kRows + r0], p1 = Ph[o * kRows + r0 + 1];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) acc[c] = fmaf(p, S[o * D + lane + 32 * c], acc[c]);
-    }
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        const int n = lane + 32 * c;
-        if (kSplitOut) {
-            const __nv_bfloat16 hi = __float2bfloat16_rn(acc[c]);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(acc[c] - __bfloat162float(hi));
-            a.WT_hi[bh * D * D + (size_t)n * D + kk] = hi;
-            a.WT_lo[bh * D * D + (size_t)n * D + kk] = lo;
-        } else {
-            a.W[bh * D * D + (size_t)kk * D + n] = acc[c];
+        for (int c = 0; c < NC; ++c) {
+            const float sv = Ss[o * D + lane + 32 * c];
+            acc[0][c] = fmaf(p0, sv, acc[0][c]);
+            acc[1][c] = fmaf(p1, sv, acc[1][c]);
         }
-        if (clean) a.S_prev[bh * D * D + (size_t)kk * D + n] = S[kk * D + n];
+    }
+    if (!kSplitOut) {
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+                a.W[bh * D * D + (size_t)(k0 + r0 + rr) * D + lane + 32 * c] = acc[rr][c];
+    } else {
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+            for (int c = 0; c < NC; ++c) Wst[(r0 + rr) * (D + 1) + lane + 32 * c] = acc[rr][c];
+        __syncthreads();
+        // WT[n][k0..k0+15] (K-major B operand of the inter-frame read), hi + lo bf16
+        for (int it = tid; it < 2 * D; it += kThreads) {
+            const int n = it >> 1, half = it & 1;
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float w0 = Wst[(half * 8 + 2 * q) * (D + 1) + n];
+                const float w1 = Wst[(half * 8 + 2 * q + 1) * (D + 1) + n];
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(w0, w1);
+                const __nv_bfloat162 lv = __floats2bfloat162_rn(w0 - __low2float(hv), w1 - __high2float(hv));
+                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
+                lo[q] = *reinterpret_cast<const uint32_t*>(&lv);
+            }
+            const size_t off = bh * D * D + (size_t)n * D + k0 + half * 8;
+            *reinterpret_cast<uint4*>(a.WT_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(a.WT_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+    if (clean) {
+        float4* dst = reinterpret_cast<float4*>(a.S_prev + bh * D * D + (size_t)k0 * D);
+        for (int i = tid; i < kRows * D / 4; i += kThreads)
+            dst[i] = reinterpret_cast<const float4*>(Ss + k0 * D)[i];
     }
 }
 
@@ -282,71 +325,88 @@ __global__ void __launch_bounds__(kThreads, 1) partials_kernel(LayerArgs a) {
 }
 
 // ---------------------------------------------------------------- update apply
-// grid (D/8, H, B); warp w updates row i = 8x + w of S, columns lane + 32c.
-template <int D>
+// grid (D/16, H, B): block x updates rows i0..i0+15 of S.  S_{N-1}, phi_v^T and
+// the block's rows of sum G and sum P are staged in shared memory; each warp
+// owns two rows, every lane the columns lane + 32c.
+template <int D, typename TIO>
 struct ApplySmem {
-    static constexpr size_t bytes = sizeof(float) * (D * (D + 1) + 2 * 8 * D + kThreads);
+    static constexpr size_t bytes = sizeof(float) * (D * D + kRows * 2 * D + kThreads) +
+                                    sizeof(TIO) * D * (D + 2);
 };
 
 template <int D, typename TIO>
 __global__ void __launch_bounds__(kThreads) apply_kernel(LayerArgs a) {
     constexpr int NC = D / 32;
     extern __shared__ float smem[];
-    float* phivT = smem;                   // [D][D+1]: phivT[o][j] = phi_v[j][o]
-    float* Gi = phivT + D * (D + 1);       // [8][D]
-    float* Pi = Gi + 8 * D;                // [8][D]
-    float* red = Pi + 8 * D;               // [kThreads]
-    const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * 8;
+    float* Ss = smem;                          // [D][D]       S_{N-1}
+    float* GP = Ss + D * D;                    // [16][2D]     rows of sum G | sum P
+    float* red = GP + kRows * 2 * D;           // [kThreads]
+    TIO* PvT = (TIO*)(red + kThreads);         // [D][D+2]     PvT[o][j] = phi_v[j][o]
+    const int b = blockIdx.z, h = blockIdx.y, i0 = blockIdx.x * kRows;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = a.T;
     const size_t bh = (size_t)b * a.H + h;
 
-    // alpha = mean_t sigmoid(g_t), fixed-order tree reduction
     float sg = 0.f;
     for (int t = tid; t < T; t += kThreads) sg += sigmoidf_(a.gate_logits[bh * T + t]);
     red[tid] = sg;
+    const float4* S4 = reinterpret_cast<const float4*>(a.S_prev + bh * D * D);
+    for (int i = tid; i < D * D / 4; i += kThreads) reinterpret_cast<float4*>(Ss)[i] = S4[i];
     const TIO* pv = (const TIO*)a.phi_v + (size_t)h * D * D;
-    for (int i = tid; i < D * D; i += kThreads) phivT[(i % D) * (D + 1) + i / D] = to_f32(pv[i]);
-    for (int i = tid; i < 8 * D; i += kThreads) {
-        const int r = i / D, m = i % D;
-        float g = 0.f, p = 0.f;
-        for (int s = 0; s < a.nsplit; ++s) {
-            const float* src = a.partials + ((bh * a.nsplit + s) * D + i0 + r) * (size_t)2 * D;
-            g += src[m];
-            p += src[D + m];
+    for (int i = tid; i < D * D; i += kThreads) PvT[(i % D) * (D + 2) + i / D] = pv[i];
+    {   // fixed-order sum over the token splits; all loads of a split in flight together
+        constexpr int PER = kRows * 2 * D / kThreads;
+        float acc[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q) acc[q] = 0.f;
+        const float* base = a.partials + (bh * a.nsplit * D + i0) * (size_t)2 * D;
+        for (int sp = 0; sp < a.nsplit; ++sp) {
+            const float* src = base + (size_t)sp * D * 2 * D;
+#pragma unroll
+            for (int q = 0; q < PER; ++q) acc[q] += src[tid + q * kThreads];
         }
-        Gi[i] = g;
-        Pi[i] = p;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) GP[tid + q * kThreads] = acc[q];
     }
     __syncthreads();
-    for (int s = kThreads / 2; s > 0; s >>= 1) {
-        if (tid < s) red[tid] += red[tid + s];
+    for (int st = kThreads / 2; st > 0; st >>= 1) {
+        if (tid < st) red[tid] += red[tid + st];
         __syncthreads();
     }
     const float alpha = red[0] / (float)T;
 
-    const float* Sp = a.S_prev + bh * D * D;
-    const int i = i0 + warp;
-    float acc[NC];
+    const int r0 = 2 * warp;
+    float acc[2][NC];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) acc[c] = alpha * Sp[(size_t)i * D + lane + 32 * c];
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) acc[rr][c] = alpha * Ss[(i0 + r0 + rr) * D + lane + 32 * c];
+    const float* G0 = GP + r0 * 2 * D;
+    const float* G1 = G0 + 2 * D;
+#pragma unroll 4
     for (int o = 0; o < D; ++o) {
-        const float p = Pi[warp * D + o];
-        const float g = Gi[warp * D + o];
+        const float p0 = G0[D + o], p1 = G1[D + o];
+        const float g0 = G0[o], g1 = G1[o];
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             const int j = lane + 32 * c;
-            acc[c] = fmaf(p, phivT[o * (D + 1) + j], acc[c]);
-            acc[c] = fmaf(-g, Sp[(size_t)o * D + j], acc[c]);
+            const float f = to_f32(PvT[o * (D + 2) + j]);
+            const float sv = Ss[o * D + j];
+            acc[0][c] = fmaf(p0, f, acc[0][c]);
+            acc[1][c] = fmaf(p1, f, acc[1][c]);
+            acc[0][c] = fmaf(-g0, sv, acc[0][c]);
+            acc[1][c] = fmaf(-g1, sv, acc[1][c]);
         }
     }
     bool bad = false;
     float* S = a.state + bh * D * D;
 #pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        S[(size_t)i * D + lane + 32 * c] = acc[c];
-        bad |= !isfinite(acc[c]);
-    }
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            S[(size_t)(i0 + r0 + rr) * D + lane + 32 * c] = acc[rr][c];
+            bad |= !isfinite(acc[rr][c]);
+        }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, FLAG_NONFINITE);
 }
 

@@ -195,12 +195,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             for (int c = 0; c < 4; ++c) tmem_ld32(tS0 + s * 128 + lrow + c * 32, x + c * 32);
             tmem_ld_wait();
             const int valid = T - j * kTile;
-            float mx = -INFINITY;
+            if (valid < kTile) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                x[i] = (i < valid) ? x[i] * scale : -INFINITY;
-                mx = fmaxf(mx, x[i]);
+                for (int i = 0; i < 128; ++i)
+                    if (i >= valid) x[i] = -INFINITY;
             }
+            // row max of the raw scores: eight independent chains, then a tree
+            float m8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+            for (int i = 8; i < 128; i += 8)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[i + k]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale;
             if (j == 0) {
                 m = mx;
             } else if (mx > m + 8.0f) {
@@ -223,31 +232,35 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tmem_st_wait();
                 m = mx;
             }
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                x[i] = ex2(x[i] - m);
-                sum += x[i];
-            }
-            l += sum;
+            const float neg_m = -m;
             if (j >= 2) {
                 ok = __all_sync(0xffffffffu,
                                 mbar_wait(&bars[B_PVDONE + s], ((j >> 1) + 1) & 1, abort_word, a.flags));
                 if (!ok) break;
             }
             uint8_t* P = smem + P0 + s * kTileBytes;
+            float sum8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const float* v = x + hf * 64 + c * 8;
+                    float e[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        e[k] = ex2(fmaf(v[k], scale, neg_m));
+                        sum8[k] += e[k];
+                    }
                     uint4 w;
-                    w.x = pack_bf16(v[0], v[1]);
-                    w.y = pack_bf16(v[2], v[3]);
-                    w.z = pack_bf16(v[4], v[5]);
-                    w.w = pack_bf16(v[6], v[7]);
+                    w.x = pack_bf16(e[0], e[1]);
+                    w.y = pack_bf16(e[2], e[3]);
+                    w.z = pack_bf16(e[4], e[5]);
+                    w.w = pack_bf16(e[6], e[7]);
                     *reinterpret_cast<uint4*>(P + hf * kHalf + sw128_offset(r, c)) = w;
                 }
+            l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + s]);
