@@ -8,7 +8,7 @@
 namespace hyb {
 
 // Device status flags, kept in the first word of the caller's workspace.
-enum : unsigned { FLAG_NONFINITE = 1u, FLAG_TIMEOUT = 2u };
+enum : unsigned { FLAG_NONFINITE = 1u, FLAG_TIMEOUT = 2u, FLAG_INTERNAL = 4u };
 
 constexpr int kNumSMs = 148;          // B200
 constexpr int kUpdateTile = 128;      // tokens per key-tile of the state update
@@ -37,6 +37,7 @@ struct LayerArgs {
     __nv_bfloat16* WT_hi;      // bf16 [BH][D][D]: (phi_q^T S)^T, high part (tensor path)
     __nv_bfloat16* WT_lo;      // bf16 [BH][D][D]: low part
     float* S_prev;             // fp32 [BH][D][D]: copy of S_{N-1} (clean pass)
+    __nv_bfloat16* phivT;      // bf16 [H][D][D]: phi_v transposed (tensor path, clean pass)
     float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
     int nsplit;
     int split_tokens;

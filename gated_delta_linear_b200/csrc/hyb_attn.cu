@@ -45,11 +45,14 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     if (elems >= 2147483647.0) return HYB_ERR_UNSUPPORTED;
     p->D = D;
     p->bf16 = bf16;
-    // token splits of the state update: enough (b,h,split) blocks to cover the
-    // SMs, each split a whole number of 128-token tiles
+    // token splits of the state update, each a whole number of 128-token tiles.
+    // Tensor path: one cluster of at most 8 CTAs per (b, h), splits reduced in
+    // distributed shared memory (no partials in the workspace).  fp32 path:
+    // enough (b, h, split) blocks to cover the SMs, partials in the workspace.
     const int BH = d->B * d->H;
     const int ntiles = (d->T + kUpdateTile - 1) / kUpdateTile;
-    int want = (kNumSMs + BH - 1) / BH;
+    int want = bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH;
+    if (bf16 && want > tc::kMaxClusterRanks) want = tc::kMaxClusterRanks;
     if (want > ntiles) want = ntiles;
     if (want < 1) want = 1;
     const int tiles_per_split = (ntiles + want - 1) / want;
@@ -59,12 +62,14 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     p->off_W = kStatusBytes;
     p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
     p->off_part = align_up(p->off_Sprev + hh * sizeof(float), 256);
-    p->total = align_up(p->off_part + hh * 2 * p->nsplit * sizeof(float), 256);
+    // fp32 path: split partials; tensor path: phi_v^T per head
+    const size_t part_bytes = bf16 ? (size_t)d->H * D * D * 2 : hh * 2 * p->nsplit * sizeof(float);
+    p->total = align_up(p->off_part + part_bytes, 256);
     return HYB_OK;
 }
 
 // ---- optional kernel timing -------------------------------------------------
-enum { K_PREP = 0, K_ATTN = 1, K_PARTIALS = 2, K_APPLY = 3 };
+enum { K_PREP = 0, K_ATTN = 1, K_UPDATE = 2, K_APPLY = 3 };
 
 struct Timing {
     bool on = false;
@@ -130,7 +135,7 @@ cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
     e = timed(K_ATTN, st, [&] { simt::attn_kernel<D, TIO><<<agrid, simt::kThreads, attn_smem, st>>>(a); });
     if (e != cudaSuccess) return e;
     if (clean) {
-        e = timed(K_PARTIALS, st, [&] {
+        e = timed(K_UPDATE, st, [&] {
             simt::partials_kernel<D, TIO><<<dim3(a.nsplit, a.H, a.B), simt::kThreads, ps, st>>>(a);
         });
         if (e != cudaSuccess) return e;
@@ -176,16 +181,13 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
 
 cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     using bf16 = __nv_bfloat16;
-    static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_part[kMaxDevices],
-        done_apply[kMaxDevices];
+    static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
     constexpr int D = 128;
     cudaError_t e;
-    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(tc::partials_kernel, tc::upd::SMEM, done_part)) != cudaSuccess) return e;
     const size_t prep_smem = simt::PrepSmem<D>::bytes;
-    const size_t apply_smem = simt::ApplySmem<D, bf16>::bytes;
     if ((e = opt_in_smem(simt::prep_kernel<D, bf16, true>, prep_smem, done_prep)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(simt::apply_kernel<D, bf16>, apply_smem, done_apply)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
     const uint64_t row_bytes = (uint64_t)a.H * D * 2;
     const uint64_t bh = (uint64_t)a.B * a.H;
     CUtensorMap tq, tk, tv, tw, tphik;
@@ -206,15 +208,27 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     });
     if (e != cudaSuccess) return e;
     if (clean) {
-        e = timed(K_PARTIALS, st, [&] {
-            tc::partials_kernel<<<dim3(a.nsplit, a.H, a.B), tc::upd::kThreads, tc::upd::SMEM, st>>>(a, tk, tv,
-                                                                                                  tphik);
-        });
+        // one cluster of nsplit CTAs per (b, h)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.nsplit, a.H, a.B);
+        cfg.blockDim = dim3(tc::upd::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = tc::upd::SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = a.nsplit;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        // programmatic dependent of the attention kernel: may run on the SMs its
+        // last wave leaves idle (it reads only inputs and prep's outputs)
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        cudaError_t le = cudaSuccess;
+        e = timed(K_UPDATE, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik); });
         if (e != cudaSuccess) return e;
-        e = timed(K_APPLY, st, [&] {
-            simt::apply_kernel<D, bf16><<<rows, simt::kThreads, apply_smem, st>>>(a);
-        });
-        if (e != cudaSuccess) return e;
+        if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -266,6 +280,7 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.WT_lo = a.WT_hi + (size_t)a.B * a.H * p.D * p.D;
     a.S_prev = (float*)(ws + p.off_Sprev);
     a.partials = (float*)(ws + p.off_part);
+    a.phivT = (__nv_bfloat16*)(ws + p.off_part);
     a.nsplit = p.nsplit;
     a.split_tokens = p.split_tokens;
 
@@ -317,6 +332,7 @@ hyb_status hyb_attn_get_device_status(const void* workspace, void* stream) {
     if (cudaMemcpy(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess)
         return HYB_ERR_CUDA;
     if (flags && cudaMemset((void*)workspace, 0, sizeof(flags)) != cudaSuccess) return HYB_ERR_CUDA;
+    if (flags & FLAG_INTERNAL) return HYB_ERR_CUDA;
     if (flags & FLAG_TIMEOUT) return HYB_ERR_TIMEOUT;
     if (flags & FLAG_NONFINITE) return HYB_WARN_NONFINITE;
     return HYB_OK;
@@ -376,8 +392,8 @@ hyb_status hyb_attn_timing_end(hyb_attn_timing* out) {
 }
 
 const char* hyb_attn_kernel_name(int kernel) {
-    static const char* names[HYB_NUM_KERNELS] = {"prep", "intra_frame_attention",
-                                                 "delta_update_partials", "delta_update_apply"};
+    static const char* names[HYB_NUM_KERNELS] = {"prep", "intra_frame_attention", "delta_update",
+                                                 "delta_update_apply"};
     return (kernel >= 0 && kernel < HYB_NUM_KERNELS) ? names[kernel] : nullptr;
 }
 

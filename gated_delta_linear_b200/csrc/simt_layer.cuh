@@ -46,10 +46,27 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
     const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * kRows;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
-    const float4* S4 = reinterpret_cast<const float4*>(a.state + bh * D * D);
-    for (int i = tid; i < D * D / 4; i += kThreads) reinterpret_cast<float4*>(Ss)[i] = S4[i];
-    const TIO* phiq = (const TIO*)a.phi_q + (size_t)h * D * D;
-    for (int i = tid; i < D * kRows; i += kThreads) Ph[i] = to_f32(phiq[(i / kRows) * D + k0 + i % kRows]);
+    // all loads of a thread are issued before any shared-memory store: the
+    // stores go through generic pointers, which would otherwise serialise them
+    {
+        const float4* S4 = reinterpret_cast<const float4*>(a.state + bh * D * D);
+        constexpr int NS = D * D / 4 / kThreads;
+        float4 sv[NS];
+#pragma unroll
+        for (int u = 0; u < NS; ++u) sv[u] = S4[tid + u * kThreads];
+        const TIO* phiq = (const TIO*)a.phi_q + (size_t)h * D * D;
+        constexpr int NP = D * kRows / kThreads;
+        float pv[NP];
+#pragma unroll
+        for (int u = 0; u < NP; ++u) {
+            const int i = tid + u * kThreads;
+            pv[u] = to_f32(phiq[(i / kRows) * D + k0 + i % kRows]);
+        }
+#pragma unroll
+        for (int u = 0; u < NS; ++u) reinterpret_cast<float4*>(Ss)[tid + u * kThreads] = sv[u];
+#pragma unroll
+        for (int u = 0; u < NP; ++u) Ph[tid + u * kThreads] = pv[u];
+    }
     __syncthreads();
     const int r0 = 2 * warp;
     float acc[2][NC];
@@ -99,6 +116,27 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
         float4* dst = reinterpret_cast<float4*>(a.S_prev + bh * D * D + (size_t)k0 * D);
         for (int i = tid; i < kRows * D / 4; i += kThreads)
             dst[i] = reinterpret_cast<const float4*>(Ss + k0 * D)[i];
+    }
+    if constexpr (kSplitOut) {
+        if (clean && b == 0) {
+            // rows k0..k0+15 of phi_v^T (PvT[o][j] = phi_v[j][o]) for the tensor-path update
+            __syncthreads();  // done reading Wst
+            __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(Wst);  // [16][D+8]
+            const __nv_bfloat16* pv = (const __nv_bfloat16*)a.phi_v + (size_t)h * D * D;
+            for (int it = tid; it < 2 * D; it += kThreads) {
+                const int j = it >> 1, half = it & 1;
+                const uint4 v = *reinterpret_cast<const uint4*>(pv + (size_t)j * D + k0 + half * 8);
+                const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) stage[(half * 8 + q) * (D + 8) + j] = e[q];
+            }
+            __syncthreads();
+            for (int it = tid; it < kRows * D / 8; it += kThreads) {
+                const int o = it / (D / 8), c = it % (D / 8);
+                *reinterpret_cast<uint4*>(a.phivT + (size_t)h * D * D + (size_t)(k0 + o) * D + c * 8) =
+                    *reinterpret_cast<const uint4*>(stage + o * (D + 8) + c * 8);
+            }
+        }
     }
 }
 

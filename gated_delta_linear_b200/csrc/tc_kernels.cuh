@@ -13,16 +13,27 @@
 // by W = phi_q^T S_{N-1} (passed as a two-term bf16 split W_hi + W_lo), so the
 // inter-frame read lands in TMEM next to the softmax accumulator and the
 // epilogue writes out = O_intra + O_inter once.
-//   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
-//                 [384,512) O_inter.
-//   Shared memory: Q 32 KB | K 2 x 32 KB | V 2 x 32 KB | P 2 x 32 KB (the P
-//                 buffers hold W_hi / W_lo until the first softmax).
+//   TMEM columns: [0,128) S (after the key loop: O_inter), [128,256) O,
+//                 [256,320) P buffer 0, [320,384) P buffer 1, [384,448) Q.
+//                 P and Q are bf16, two per 32-bit column, and feed the MMAs
+//                 as A operands, so per key tile shared memory only carries K
+//                 and V.  As soon as both softmax halves have read S_j, the MMA
+//                 warp issues S_{j+1} into the same columns, so the next tile's
+//                 scores are computed while the softmax exponentiates this one.
+//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Q moves to TMEM at
+//                 the start; W_hi then takes its buffer and W_lo a V stage the
+//                 key loop no longer needs, and O_inter = Q W_hi + Q W_lo is
+//                 computed while the softmax works on the last tile.
+//   Every CTA signals at entry that the next kernel (the delta update, which
+//   reads none of this kernel's outputs) may start on idle SMs.
 //
-// delta_update_partials: one CTA per (token split, head, batch).  Per 128-token
-// tile: K~ = K phi_k^T on the tensor core, row L2-normalisation and beta in
-// registers, then G += (beta K')^T K' and P += (beta K')^T V as MN-major
-// contractions over the tokens, with beta K' and K' split into bf16 hi + lo
-// (G takes hi*hi + hi*lo + lo*hi, P takes hi*V + lo*V; V is exact in bf16).
+// delta_update: one cluster per (head, batch), one CTA per token split.  Per
+// 128-token tile: K~ = K phi_k^T on the tensor core, row L2-normalisation and
+// beta in registers, then G += (beta K')^T K' and P += (beta K')^T V as
+// MN-major contractions over the tokens, with beta K' and K' split into bf16
+// hi + lo (G takes hi*hi + hi*lo + lo*hi, P takes hi*V + lo*V; V is exact in
+// bf16); the splits are then reduced through distributed shared memory and
+// the update is applied in fp32 (see the kernel's comment).
 #pragma once
 
 #include "common.cuh"
@@ -36,18 +47,23 @@ using namespace sm100;
 constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr uint32_t kHalf = kTileBytes / 2;      // one 128 x 64 TMA box
+constexpr int kMaxClusterRanks = 8;             // token splits per (b, h) in the update
 
 // ============================================================== attention
 namespace attn {
+constexpr int kStages = 3;                     // K and V ring depth
 constexpr uint32_t Q = 0;
 constexpr uint32_t K0 = Q + kTileBytes;
-constexpr uint32_t V0 = K0 + 2 * kTileBytes;
-constexpr uint32_t P0 = V0 + 2 * kTileBytes;
-constexpr uint32_t BAR = P0 + 2 * kTileBytes;
-constexpr uint32_t SMEM = 1024 + BAR + 256;  // + alignment slack + barriers
-constexpr int kThreads = 192;
-enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_PFULL = 11,
-       B_PVDONE = 13, B_COUNT = 15 };
+constexpr uint32_t V0 = K0 + kStages * kTileBytes;
+constexpr uint32_t BAR = V0 + kStages * kTileBytes;
+constexpr uint32_t XCHG = BAR + 256;          // softmax pair exchange: [2][2][128] floats
+constexpr uint32_t XOK = XCHG + 2048;         // and [2][2][128] wait results (bytes)
+constexpr uint32_t SMEM = XOK + 512;          // 232,192 B
+constexpr int kSoftmaxThreads = 256;           // warps 0-7
+constexpr int kLoadWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
+enum { B_Q = 0, B_QTMEM = 1, B_W = 2, B_OIDONE = 3, B_KFULL = 4, B_KEMPTY = 7, B_VFULL = 10,
+       B_VEMPTY = 13, B_SFULL = 16, B_SREAD = 17, B_PFULL = 18, B_PVDONE = 20, B_COUNT = 22 };
 }  // namespace attn
 
 // K-major operand, 128 rows x 128 bf16 stored as two 64-column swizzled boxes:
@@ -65,13 +81,23 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_w) {
     using namespace attn;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // 128B-swizzled tiles need a 1024-byte aligned base (the dynamic window starts
+    // after the 1 KB reserved block); report and leave if it is not
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
+        return;
+    }
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
     volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+    float* xchg = (float*)(smem + XCHG);    // [2 parity][2 halves][128 rows] row maxima, then row sums
+    uint8_t* xok = smem + XOK;              // [2 parity][2 halves][128 rows] wait results
 
+    // the delta update of this pass does not read anything this kernel writes:
+    // it may start on SMs this grid leaves idle
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T;
@@ -80,18 +106,22 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int bh = b * a.H + h;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_PFULL || i == B_PFULL + 1 ? 128 : 1);
+        for (int i = 0; i < B_COUNT; ++i)
+            mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1 || i == B_SREAD || i == B_QTMEM)
+                                    ? kSoftmaxThreads
+                                    : 1);
         *abort_word = 0;
         fence_mbar_init();
     }
-    if (warp == 5) tmem_alloc(tmem_slot, 512);
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tO = tmem + 256, tOI = tmem + 384;
+    const uint32_t tS = tmem, tO = tmem + 128, tP0 = tmem + 256, tQ = tmem + 384;
+    const uint32_t tOI = tS;  // O_inter reuses the S columns after the last softmax read
 
-    if (warp == 4) {
+    if (warp == kLoadWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
@@ -99,77 +129,91 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_w);
             const int xh = h * 128;
-            mbar_expect_tx(&bars[B_Q], 3 * kTileBytes);
+            mbar_expect_tx(&bars[B_Q], kTileBytes);
             tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0, b);
             tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
+            bool ok = true;
+            for (int j = 0; j < n && ok; ++j) {
+                const int st = j % kStages;
+                const uint32_t par = ((j / kStages) + 1) & 1;
+                if (j >= kStages && !(ok = mbar_wait(&bars[B_KEMPTY + st], par, abort_word, a.flags))) break;
+                mbar_expect_tx(&bars[B_KFULL + st], kTileBytes);
+                tma_load_3d(sb + K0 + st * kTileBytes, &tm_k, &bars[B_KFULL + st], xh, j * kTile, b);
+                tma_load_3d(sb + K0 + st * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + st], xh + 64, j * kTile, b);
+                if (j >= kStages && !(ok = mbar_wait(&bars[B_VEMPTY + st], par, abort_word, a.flags))) break;
+                mbar_expect_tx(&bars[B_VFULL + st], kTileBytes);
+                tma_load_3d(sb + V0 + st * kTileBytes, &tm_v, &bars[B_VFULL + st], xh, j * kTile, b);
+                tma_load_3d(sb + V0 + st * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + st], xh + 64, j * kTile, b);
+            }
+            // W_hi into the Q buffer once Q is in TMEM; W_lo into the V stage of
+            // tile n-3 once PV_{n-3} has read it (stage 2, never used, when n < 3)
             const int nbh = a.B * a.H;
-            tma_load_3d(sb + P0, &tm_w, &bars[B_Q], 0, 0, bh);
-            tma_load_3d(sb + P0 + kHalf, &tm_w, &bars[B_Q], 64, 0, bh);
-            tma_load_3d(sb + P0 + kTileBytes, &tm_w, &bars[B_Q], 0, 0, nbh + bh);
-            tma_load_3d(sb + P0 + kTileBytes + kHalf, &tm_w, &bars[B_Q], 64, 0, nbh + bh);
-            for (int j = 0; j < n; ++j) {
-                const int s = j & 1;
-                const uint32_t par = ((j >> 1) + 1) & 1;
-                if (j >= 2 && !mbar_wait(&bars[B_KEMPTY + s], par, abort_word, a.flags)) break;
-                mbar_expect_tx(&bars[B_KFULL + s], kTileBytes);
-                tma_load_3d(sb + K0 + s * kTileBytes, &tm_k, &bars[B_KFULL + s], xh, j * kTile, b);
-                tma_load_3d(sb + K0 + s * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + s], xh + 64, j * kTile, b);
-                if (j >= 2 && !mbar_wait(&bars[B_VEMPTY + s], par, abort_word, a.flags)) break;
-                mbar_expect_tx(&bars[B_VFULL + s], kTileBytes);
-                tma_load_3d(sb + V0 + s * kTileBytes, &tm_v, &bars[B_VFULL + s], xh, j * kTile, b);
-                tma_load_3d(sb + V0 + s * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + s], xh + 64, j * kTile, b);
+            const int wst = n >= 3 ? (n - 3) % kStages : 2;
+            if (ok) ok = mbar_wait(&bars[B_QTMEM], 0, abort_word, a.flags);
+            if (ok && n >= 3) ok = mbar_wait(&bars[B_VEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
+            if (ok) {
+                mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
+                tma_load_3d(sb + Q, &tm_w, &bars[B_W], 0, 0, bh);
+                tma_load_3d(sb + Q + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
+                tma_load_3d(sb + V0 + wst * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
+                tma_load_3d(sb + V0 + wst * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags);
+            bool ok = mbar_wait(&bars[B_QTMEM], 0, abort_word, a.flags);
             if (ok) {
-                tc_fence_after();
-                // O_inter = Q W_hi + Q W_lo
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), kmajor_desc(sb + P0, kk), ID_KK, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), kmajor_desc(sb + P0 + kTileBytes, kk), ID_KK, 1);
-                for (int j = 0; j < 2 && j < n && ok; ++j) {
-                    ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags);
-                    if (!ok) break;
+                ok = mbar_wait(&bars[B_KFULL], 0, abort_word, a.flags);
+                if (ok) {
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk),
-                                 kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK, kk > 0);
-                    mma_commit(&bars[B_SFULL + j]);
-                    mma_commit(&bars[B_KEMPTY + j]);
+                        mma_bf16_ts(tS, tQ + kk * 8, kmajor_desc(sb + K0, kk), ID_KK, kk > 0);
+                    mma_commit(&bars[B_SFULL]);
+                    mma_commit(&bars[B_KEMPTY]);
                 }
             }
             for (int j = 0; j < n && ok; ++j) {
-                const int s = j & 1;
-                const uint32_t par = (j >> 1) & 1;
-                if (!mbar_wait(&bars[B_PFULL + s], par, abort_word, a.flags)) break;
-                if (!mbar_wait(&bars[B_VFULL + s], par, abort_word, a.flags)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tO, kmajor_desc(sb + P0 + s * kTileBytes, kk),
-                             mnmajor_desc(sb + V0 + s * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
-                mma_commit(&bars[B_PVDONE + s]);
-                mma_commit(&bars[B_VEMPTY + s]);
-                if (j + 2 < n) {
-                    if (!mbar_wait(&bars[B_KFULL + s], ((j + 2) >> 1) & 1, abort_word, a.flags)) break;
+                if (j + 1 < n) {
+                    // S_{j+1} into the S columns once both halves have read S_j
+                    const int st1 = (j + 1) % kStages;
+                    if (!mbar_wait(&bars[B_SREAD], j & 1, abort_word, a.flags)) break;
+                    if (!mbar_wait(&bars[B_KFULL + st1], ((j + 1) / kStages) & 1, abort_word, a.flags)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tS0 + s * 128, kmajor_desc(sb + Q, kk),
-                                 kmajor_desc(sb + K0 + s * kTileBytes, kk), ID_KK, kk > 0);
-                    mma_commit(&bars[B_SFULL + s]);
-                    mma_commit(&bars[B_KEMPTY + s]);
+                        mma_bf16_ts(tS, tQ + kk * 8, kmajor_desc(sb + K0 + st1 * kTileBytes, kk), ID_KK, kk > 0);
+                    mma_commit(&bars[B_SFULL]);
+                    mma_commit(&bars[B_KEMPTY + st1]);
                 }
+                const int pb = j & 1, st = j % kStages;
+                if (!mbar_wait(&bars[B_PFULL + pb], (j >> 1) & 1, abort_word, a.flags)) break;
+                if (!mbar_wait(&bars[B_VFULL + st], (j / kStages) & 1, abort_word, a.flags)) break;
+                tc_fence_after();
+                // O += P_j V_j, P_j from TMEM P buffer pb
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tO, tP0 + pb * 64 + kk * 8, mnmajor_desc(sb + V0 + st * kTileBytes, kk), ID_KMN,
+                                (j > 0 || kk > 0));
+                mma_commit(&bars[B_PVDONE + pb]);
+                mma_commit(&bars[B_VEMPTY + st]);
+            }
+            // O_inter = Q W_hi + Q W_lo into the S columns, once the last S is read
+            if (ok) ok = mbar_wait(&bars[B_SREAD], (n - 1) & 1, abort_word, a.flags);
+            if (ok) ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags);
+            if (ok) {
+                tc_fence_after();
+                const int wst = n >= 3 ? (n - 3) % kStages : 2;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tOI, tQ + kk * 8, kmajor_desc(sb + Q, kk), ID_KK, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tOI, tQ + kk * 8, kmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KK, 1);
+                mma_commit(&bars[B_OIDONE]);
             }
             // drain: every MMA issued so far completes before TMEM is released
             mma_commit(&bars[B_Q]);
@@ -179,104 +223,154 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ softmax + epilogue (row r)
-        const int r = threadIdx.x;  // 0..127, TMEM lane r
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        // ------------------------------------------------ softmax + epilogue
+        // Warp w owns TMEM lanes (query rows) 32(w%4)..+31 and key half ch = w/4
+        // (keys 64ch..64ch+63 of each tile; output columns 64ch..64ch+63).  The
+        // two warps sharing rows exchange their half-row maxima through shared
+        // memory at a pair barrier every iteration; every wait result goes through
+        // the same exchange, so both warps always take the same path.
+        const int ch = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const int pair_bar = 1 + (warp & 3);
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         const float scale = a.sm_scale_log2;
         float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        float x[128];
+        // Q row r, features 64ch..64ch+63, from the swizzled TMA tile into TMEM
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags));
+        if (ok) {
+            uint32_t qv[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + ch * kHalf + sw128_offset(r, c));
+                qv[4 * c + 0] = v.x;
+                qv[4 * c + 1] = v.y;
+                qv[4 * c + 2] = v.z;
+                qv[4 * c + 3] = v.w;
+            }
+            tmem_st32u(tQ + lrow + ch * 32, qv);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[B_QTMEM]);
+        }
+        float x[64];
         for (int j = 0; j < n; ++j) {
             const int s = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + s], (j >> 1) & 1, abort_word, a.flags));
-            if (!ok) break;
-            tc_fence_after();
+            // waits of this iteration: S_j ready; P buffer s free (PV_{j-2} done)
+            bool w_ok = ok && mbar_wait(&bars[B_SFULL], j & 1, abort_word, a.flags);
+            if (j >= 2) w_ok = w_ok && mbar_wait(&bars[B_PVDONE + s], ((j >> 1) + 1) & 1, abort_word, a.flags);
+            w_ok = __all_sync(0xffffffffu, w_ok);
+            float hm = -INFINITY;
+            if (w_ok) {
+                tc_fence_after();
+                tmem_ld32(tS + lrow + ch * 64, x);
+                tmem_ld32(tS + lrow + ch * 64 + 32, x + 32);
+                tmem_ld_wait();
+                // S_j is in registers: the MMA warp may overwrite it with S_{j+1}
+                tc_fence_before();
+                mbar_arrive(&bars[B_SREAD]);
+                const int valid = T - j * kTile - ch * 64;
+                if (valid < 64) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS0 + s * 128 + lrow + c * 32, x + c * 32);
-            tmem_ld_wait();
-            const int valid = T - j * kTile;
-            if (valid < kTile) {
+                    for (int i = 0; i < 64; ++i)
+                        if (i >= valid) x[i] = -INFINITY;
+                }
+                float m8[8];
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    if (i >= valid) x[i] = -INFINITY;
+                for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+                for (int i = 8; i < 64; i += 8)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[i + k]);
+                hm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             }
-            // row max of the raw scores: eight independent chains, then a tree
-            float m8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = x[k];
-#pragma unroll
-            for (int i = 8; i < 128; i += 8)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[i + k]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale;
+            xchg[(s * 2 + ch) * 128 + r] = hm;
+            xok[(s * 2 + ch) * 128 + r] = (uint8_t)w_ok;
+            named_bar_sync(pair_bar, 64);
+            ok = w_ok && xok[(s * 2 + (ch ^ 1)) * 128 + r];
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) continue;   // keep arriving at the pair barriers until the loop ends
+            const float mx = fmaxf(hm, xchg[(s * 2 + (ch ^ 1)) * 128 + r]) * scale;
+            bool rescale = false;
             if (j == 0) {
                 m = mx;
             } else if (mx > m + 8.0f) {
-                // the running max moved by more than 2^8: rescale O (after PV_{j-1})
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + ((j - 1) & 1)], ((j - 1) >> 1) & 1,
-                                                         abort_word, a.flags));
-                if (!ok) break;
-                tc_fence_after();
-                const float f = ex2(m - mx);
-                l *= f;
-                float o[32];
+                rescale = true;
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                // the running max moved by more than 2^8: rescale this half of O (after PV_{j-1})
+                const bool pv_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + ((j - 1) & 1)],
+                                                                    ((j - 1) >> 1) & 1, abort_word, a.flags));
+                if (pv_ok) {
+                    tc_fence_after();
+                    const float f = rescale ? ex2(m - mx) : 1.0f;
+                    float o[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tO + lrow + c * 32, o);
-                    tmem_ld_wait();
+                    for (int c = 0; c < 2; ++c) {
+                        tmem_ld32(tO + lrow + ch * 64 + c * 32, o);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= f;
-                    tmem_st32(tO + lrow + c * 32, o);
+                        for (int i = 0; i < 32; ++i) o[i] *= f;
+                        tmem_st32(tO + lrow + ch * 64 + c * 32, o);
+                    }
+                    tmem_st_wait();
+                    if (rescale) {
+                        l *= f;
+                        m = mx;
+                    }
+                } else {
+                    ok = false;  // P_j is not written; the MMA warp times out on it
                 }
-                tmem_st_wait();
-                m = mx;
             }
             const float neg_m = -m;
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(&bars[B_PVDONE + s], ((j >> 1) + 1) & 1, abort_word, a.flags));
-                if (!ok) break;
-            }
-            uint8_t* P = smem + P0 + s * kTileBytes;
+            // P (bf16 pairs) into this half's 32 columns of P buffer s
+            uint32_t pk[32];
             float sum8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+            // 1 of every 8 exponentials on the FMA pipe, the rest on MUFU; the
+            // bf16 packing on the integer pipe (MUFU is the scarce pipe here)
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
+            for (int c = 0; c < 8; ++c) {
+                float e[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float* v = x + hf * 64 + c * 8;
-                    float e[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        e[k] = ex2(fmaf(v[k], scale, neg_m));
-                        sum8[k] += e[k];
-                    }
-                    uint4 w;
-                    w.x = pack_bf16(e[0], e[1]);
-                    w.y = pack_bf16(e[2], e[3]);
-                    w.z = pack_bf16(e[4], e[5]);
-                    w.w = pack_bf16(e[6], e[7]);
-                    *reinterpret_cast<uint4*>(P + hf * kHalf + sw128_offset(r, c)) = w;
+                for (int k = 0; k < 8; ++k) {
+                    const float arg = fmaf(x[c * 8 + k], scale, neg_m);
+                    e[k] = (k == 4) ? exp2_fma(arg) : ex2(arg);
+                    sum8[k] += e[k];
                 }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16_rhu(e[2 * k], e[2 * k + 1]);
+            }
             l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-            fence_async_smem();
+            tmem_st32u(tP0 + s * 64 + lrow + ch * 32, pk);
+            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&bars[B_PFULL + s]);
+            if (ok) mbar_arrive(&bars[B_PFULL + s]);
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + ((n - 1) & 1)], ((n - 1) >> 1) & 1,
-                                                        abort_word, a.flags));
-        if (ok) {
+        // epilogue: row sum from both halves (fixed order), then this half's output columns
+        bool e_ok = ok && mbar_wait(&bars[B_PVDONE + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_word, a.flags);
+        e_ok = e_ok && mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags);
+        e_ok = __all_sync(0xffffffffu, e_ok);
+        // slot n&1 was last used in iteration n-2; the partner read it before the
+        // barrier of iteration n-1, so it is free (slot (n-1)&1 may still be read)
+        const int se = n & 1;
+        xchg[(se * 2 + ch) * 128 + r] = l;
+        xok[(se * 2 + ch) * 128 + r] = (uint8_t)e_ok;
+        named_bar_sync(pair_bar, 64);
+        e_ok = e_ok && xok[(se * 2 + (ch ^ 1)) * 128 + r];
+        e_ok = __all_sync(0xffffffffu, e_ok);
+        if (e_ok) {
             tc_fence_after();
+            const float lt = xchg[(se * 2 + 0) * 128 + r] + xchg[(se * 2 + 1) * 128 + r];
             const int t = q0 + r;
-            const float inv_l = 1.0f / l;
-            const size_t row = (((size_t)b * T + t) * a.H + h) * 128;
+            const float inv_l = 1.0f / lt;
+            const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + ch * 64;
             float o[32], e[32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld32(tO + lrow + c * 32, o);
-                tmem_ld32(tOI + lrow + c * 32, e);
+            for (int c = 0; c < 2; ++c) {
+                tmem_ld32(tO + lrow + ch * 64 + c * 32, o);
+                tmem_ld32(tOI + lrow + ch * 64 + c * 32, e);
                 tmem_ld_wait();
                 if (t < T) {
                     if (a.out) {
@@ -308,11 +402,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
-// ============================================================== update partials
+// ============================================================== delta update
+// One cluster of C CTAs per (batch, head); CTA c of the cluster takes token
+// split c (a run of 128-token tiles) and accumulates its G_c = (beta K')^T K'
+// and P_c = (beta K')^T V in TMEM.  The CTAs then park [G_c | P_c] in shared
+// memory, each reduces its own band of rows over the C CTAs through
+// distributed shared memory (fixed order c = 0..C-1, so the result is
+// deterministic), and applies the update to that band:
+//   S_N[i][:] = alpha S_{N-1}[i][:] + P[i][:] phi_v^T - G[i][:] S_{N-1}
+// with alpha = mean_t sigmoid(g_t); S_{N-1} and phi_v^T come from the
+// workspace (written by the prep kernel of the same pass).
 namespace upd {
+// tile loop (1024-aligned 128B-swizzled tiles)
 constexpr uint32_t PHI = 0;
 constexpr uint32_t KT = PHI + kTileBytes;
 constexpr uint32_t VT = KT + kTileBytes;
@@ -320,45 +424,91 @@ constexpr uint32_t AH = VT + kTileBytes;
 constexpr uint32_t AL = AH + kTileBytes;
 constexpr uint32_t KH = AL + kTileBytes;
 constexpr uint32_t KL = KH + kTileBytes;
-constexpr uint32_t BAR = KL + kTileBytes;
-constexpr uint32_t SMEM = 1024 + BAR + 256;
-constexpr int kThreads = 192;
-enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_OPSFULL, B_OPSFREE, B_COUNT };
+constexpr uint32_t TILES_END = KL + kTileBytes;          // 229,376
+// after the tile loop (reuses the tile space)
+constexpr uint32_t PHIVT = 0;                             // phi_v^T bf16 [128][128]
+constexpr uint32_t SPREV = PHIVT + 128 * 128 * 2;         // S_{N-1} fp32 [128][128]
+constexpr uint32_t RED = SPREV + 128 * 128 * 4;           // [128][256] fp32, 16-byte chunks XOR-swizzled by row
+constexpr uint32_t BAR = TILES_END;                       // barriers, TMEM slot, flags, sums
+constexpr uint32_t XSS = BAR + 256;                       // [2 parity][2 halves][128 rows] floats + ok bytes
+constexpr uint32_t SMEM = XSS + 2048 + 512;               // 232,192 B
+constexpr int kNormThreads = 256;                         // warps 0-7
+constexpr int kLoadWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
+enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_OPSFULL, B_OPSFREE, B_PARK, B_COUNT };
+static_assert(RED + 128 * 256 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
+// byte offset of float4 chunk q (0..63) of row `row` in RED
+__device__ __forceinline__ uint32_t red_off(int row, int q) {
+    return (uint32_t)(row * 1024 + ((q ^ (row & 7)) << 4));
+}
 }  // namespace upd
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
+}
+
 __global__ void __launch_bounds__(upd::kThreads, 1)
-    partials_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_phik) {
+    update_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_phik) {
     using namespace upd;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {  // uniform over the grid: every CTA leaves
+        if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
+        return;
+    }
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
     volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+    float* wsum = (float*)(tmem_slot + 2);  // 10 warp partial sums + alpha
+    float* xss = (float*)(smem + XSS);      // row sums of squares exchanged between warp pairs
+    uint8_t* xok = smem + XSS + 2048;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int split = (int)cluster_ctarank();
+    const int C = (int)cluster_nctarank();
     const int T = a.T;
     const int bh = b * a.H + h;
     const int t_begin = split * a.split_tokens;
     const int t_end = min(T, t_begin + a.split_tokens);
-    const int nt = (t_end - t_begin + kTile - 1) / kTile;
+    const int nt = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_OPSFULL ? 128 : 1);
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_OPSFULL ? kNormThreads : 1);
         *abort_word = 0;
         fence_mbar_init();
     }
-    if (warp == 5) tmem_alloc(tmem_slot, 512);
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tKT = tmem, tG = tmem + 128, tP = tmem + 256;
 
-    if (warp == 4) {
-        if (lane == 0) {
+    // ------------------------------------------------------------ tile loop
+    if (warp == kLoadWarp) {
+        if (lane == 0 && nt > 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_phik);
@@ -379,8 +529,8 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
-        if (lane == 0) {
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && nt > 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_MNMN = idesc_bf16(128, 128, 1, 1);
             bool ok = mbar_wait(&bars[B_PHI], 0, abort_word, a.flags);
@@ -398,15 +548,16 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t first = (i > 0 || kk > 0);
-                    mma_bf16(tG, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + KH, kk), ID_MNMN, first);
+                    const uint32_t acc = (i > 0 || kk > 0);
+                    mma_bf16(tG, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + KH, kk), ID_MNMN, acc);
                     mma_bf16(tG, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + KL, kk), ID_MNMN, 1);
                     mma_bf16(tG, mnmajor_desc(sb + AL, kk), mnmajor_desc(sb + KH, kk), ID_MNMN, 1);
-                    mma_bf16(tP, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + VT, kk), ID_MNMN, first);
+                    mma_bf16(tP, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + VT, kk), ID_MNMN, acc);
                     mma_bf16(tP, mnmajor_desc(sb + AL, kk), mnmajor_desc(sb + VT, kk), ID_MNMN, 1);
                 }
                 mma_commit(&bars[B_OPSFREE]);
             }
+            // drain: every MMA issued so far completes before the tile space is reused
             mma_commit(&bars[B_PHI]);
             uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(smem_u32(&bars[B_PHI]), 1) && globaltimer_ns() - t0 < kWaitNs) {
@@ -414,94 +565,214 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         }
         __syncwarp();
     } else {
-        const int r = threadIdx.x;  // token row within the tile, TMEM lane r
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        // Warps w and w+4 share token rows (TMEM lanes 32(w%4)..+31); warp w/4 = half
+        // takes feature columns 64*half..64*half+63.  The pair exchanges its half
+        // sums of squares (and wait results) at a named barrier every tile.
+        const int half = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const int pair_bar = 1 + (warp & 3);
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
-        float x[128];
+        float x[64];
         for (int i = 0; i < nt; ++i) {
-            const uint32_t par = i & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KTFULL], par, abort_word, a.flags));
-            if (!ok) break;
-            tc_fence_after();
+            const int s = i & 1;
+            bool w_ok = ok && mbar_wait(&bars[B_KTFULL], i & 1, abort_word, a.flags);
+            if (i > 0) w_ok = w_ok && mbar_wait(&bars[B_OPSFREE], (i - 1) & 1, abort_word, a.flags);
+            w_ok = __all_sync(0xffffffffu, w_ok);
+            float ssh = 0.f;
+            if (w_ok) {
+                tc_fence_after();
+                tmem_ld32(tKT + lrow + half * 64, x);
+                tmem_ld32(tKT + lrow + half * 64 + 32, x + 32);
+                tmem_ld_wait();
+                float ss8[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tKT + lrow + c * 32, x + c * 32);
-            tmem_ld_wait();
+                for (int k = 0; k < 8; ++k) ss8[k] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) ss8[c & 7] = fmaf(x[c], x[c], ss8[c & 7]);
+                ssh = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
+            }
+            xss[(s * 2 + half) * 128 + r] = ssh;
+            xok[(s * 2 + half) * 128 + r] = (uint8_t)w_ok;
+            named_bar_sync(pair_bar, 64);
+            ok = __all_sync(0xffffffffu, w_ok && xok[(s * 2 + (half ^ 1)) * 128 + r]);
+            if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
+            const float ss = xss[(s * 2 + 0) * 128 + r] + xss[(s * 2 + 1) * 128 + r];
             const int tok = t_begin + i * kTile + r;
             const bool valid = tok < t_end;
-            float ss = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) ss = fmaf(x[c], x[c], ss);
             const float inv = valid ? 1.0f / sqrtf(ss + a.l2_eps) : 0.f;
             const float beta = valid ? sigmoidf_(a.beta_logits[(size_t)bh * T + tok]) : 0.f;
-            if (i > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OPSFREE], (i - 1) & 1, abort_word, a.flags));
-                if (!ok) break;
-            }
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
+            for (int c = 0; c < 8; ++c) {
+                uint32_t ah[4], al[4], kh[4], kl[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t ah[4], al[4], kh[4], kl[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int col = hf * 64 + c * 8 + 2 * q;
-                        float k0 = x[col] * inv, k1 = x[col + 1] * inv;
-                        float a0 = k0 * beta, a1 = k1 * beta;
-                        __nv_bfloat162 khv = __floats2bfloat162_rn(k0, k1);
-                        __nv_bfloat162 ahv = __floats2bfloat162_rn(a0, a1);
-                        kh[q] = *reinterpret_cast<uint32_t*>(&khv);
-                        ah[q] = *reinterpret_cast<uint32_t*>(&ahv);
-                        kl[q] = pack_bf16(k0 - __low2float(khv), k1 - __high2float(khv));
-                        al[q] = pack_bf16(a0 - __low2float(ahv), a1 - __high2float(ahv));
-                    }
-                    const uint32_t off = hf * kHalf + sw128_offset(r, c);
-                    *reinterpret_cast<uint4*>(smem + AH + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-                    *reinterpret_cast<uint4*>(smem + AL + off) = make_uint4(al[0], al[1], al[2], al[3]);
-                    *reinterpret_cast<uint4*>(smem + KH + off) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-                    *reinterpret_cast<uint4*>(smem + KL + off) = make_uint4(kl[0], kl[1], kl[2], kl[3]);
+                for (int q = 0; q < 4; ++q) {
+                    const int col = c * 8 + 2 * q;
+                    const float k0 = x[col] * inv, k1 = x[col + 1] * inv;
+                    const float a0 = k0 * beta, a1 = k1 * beta;
+                    const __nv_bfloat162 khv = __floats2bfloat162_rn(k0, k1);
+                    const __nv_bfloat162 ahv = __floats2bfloat162_rn(a0, a1);
+                    kh[q] = *reinterpret_cast<const uint32_t*>(&khv);
+                    ah[q] = *reinterpret_cast<const uint32_t*>(&ahv);
+                    kl[q] = pack_bf16(k0 - __low2float(khv), k1 - __high2float(khv));
+                    al[q] = pack_bf16(a0 - __low2float(ahv), a1 - __high2float(ahv));
                 }
+                const uint32_t off = half * kHalf + sw128_offset(r, c);
+                *reinterpret_cast<uint4*>(smem + AH + off) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+                *reinterpret_cast<uint4*>(smem + AL + off) = make_uint4(al[0], al[1], al[2], al[3]);
+                *reinterpret_cast<uint4*>(smem + KH + off) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+                *reinterpret_cast<uint4*>(smem + KL + off) = make_uint4(kl[0], kl[1], kl[2], kl[3]);
+            }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_OPSFULL]);
         }
         if (ok && nt > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OPSFREE], (nt - 1) & 1, abort_word, a.flags));
-        if (ok) {
-            tc_fence_after();
-            // row r of G and P (TMEM lane = output row i)
-            float* dst = a.partials + (((size_t)bh * a.nsplit + split) * 128 + r) * 256;
-            float v[32];
-            for (int c = 0; c < 4; ++c) {
-                if (nt > 0) {
-                    tmem_ld32(tG + lrow + c * 32, v);
-                    tmem_ld_wait();
-                } else {
+    }
+    // ------------------------------------------------------------ park [G | P]; stage S_{N-1}, phi_v^T
+    tc_fence_before();
+    __syncthreads();  // every MMA has completed (or timed out): the tile space is free
+    tc_fence_after();
+    if (threadIdx.x == kLoadWarp * 32) {
+        mbar_expect_tx(&bars[B_PARK], 128 * 128 * 2 + 128 * 128 * 4);
+        bulk_load(sb + PHIVT, a.phivT + (size_t)h * 128 * 128, 128 * 128 * 2, &bars[B_PARK]);
+        bulk_load(sb + SPREV, a.S_prev + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
+    }
+    {
+        float sg = 0.f;
+        for (int t = threadIdx.x; t < T; t += kThreads) sg += sigmoidf_(a.gate_logits[(size_t)bh * T + t]);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
-                }
+        for (int o = 16; o > 0; o >>= 1) sg += __shfl_xor_sync(0xffffffffu, sg, o);
+        if (lane == 0) wsum[warp] = sg;
+    }
+    if (warp < 8) {
+        // this warp's rows, columns [64 half, 64 half + 64) of G and of P
+        const int half = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        float v[32];
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    reinterpret_cast<float4*>(dst + c * 32)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int c = 0; c < 4; ++c) {  // c: G lo, G hi, P lo, P hi (32 columns each)
+            const uint32_t src = (c < 2 ? tG : tP) + lrow + half * 64 + (c & 1) * 32;
+            if (nt > 0) {
+                tmem_ld32(src, v);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) v[q] = 0.f;
             }
-            for (int c = 0; c < 4; ++c) {
-                if (nt > 0) {
-                    tmem_ld32(tP + lrow + c * 32, v);
-                    tmem_ld_wait();
-                } else {
+            const int q0 = (c >> 1) * 32 + half * 16 + (c & 1) * 8;  // first float4 chunk
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    reinterpret_cast<float4*>(dst + 128 + c * 32)[q] =
-                        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            }
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(smem + RED + red_off(row, q0 + q)) =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
     }
-    tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) t += wsum[w];
+        wsum[10] = t / (float)T;
+    }
+    cluster_sync();  // every CTA of the cluster has parked its [G | P]
+
+    // ------------------------------------------------------------ reduce this CTA's band of rows
+    const int band = (128 + C - 1) / C;
+    const int r0 = min(128, split * band), r1 = min(128, r0 + band);
+    {
+        const int items = (r1 - r0) * 64;
+        // two items per step, all their C remote loads in flight together
+        for (int it = threadIdx.x; it < items; it += 2 * kThreads) {
+            const int it2 = it + kThreads;
+            const bool second = it2 < items;
+            const uint32_t off0 = red_off(r0 + it / 64, it % 64);
+            const uint32_t off1 = second ? red_off(r0 + it2 / 64, it2 % 64) : off0;
+            float4 v0[kMaxClusterRanks], v1[kMaxClusterRanks];
+#pragma unroll
+            for (int c = 0; c < kMaxClusterRanks; ++c)
+                if (c < C) {
+                    v0[c] = ld_cluster_f4(sb + RED + off0, (uint32_t)c);
+                    v1[c] = ld_cluster_f4(sb + RED + off1, (uint32_t)c);
+                }
+            float4 s0 = v0[0], s1 = v1[0];
+#pragma unroll
+            for (int c = 1; c < kMaxClusterRanks; ++c)
+                if (c < C) {
+                    s0.x += v0[c].x; s0.y += v0[c].y; s0.z += v0[c].z; s0.w += v0[c].w;
+                    s1.x += v1[c].x; s1.y += v1[c].y; s1.z += v1[c].z; s1.w += v1[c].w;
+                }
+            *reinterpret_cast<float4*>(smem + RED + off0) = s0;
+            if (second) *reinterpret_cast<float4*>(smem + RED + off1) = s1;
+        }
+    }
+    const bool park_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PARK], 0, abort_word, a.flags));
+    __syncthreads();
+
+    // ------------------------------------------------------------ apply to the band
+    if (warp < 8 && park_ok) {
+        const int j = threadIdx.x & 127;  // output column
+        const int rs = threadIdx.x >> 7;  // this thread takes rows r0 + rs, r0 + rs + 2, ...
+        const float alpha = wsum[10];
+        const float* Sp = reinterpret_cast<const float*>(smem + SPREV);
+        const __nv_bfloat16* Pt = reinterpret_cast<const __nv_bfloat16*>(smem + PHIVT);
+        float* S = a.state + (size_t)bh * 128 * 128;
+        bool bad = false;
+        for (int rc = r0 + rs; rc < r1; rc += 16) {
+            // rows rc, rc + 2, ..., rc + 14; rows at or past r1 are computed on
+            // clamped (valid) data and discarded
+            int rowi[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rowi[i] = min(rc + 2 * i, 127);
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = alpha * Sp[rowi[i] * 128 + j];
+#pragma unroll 2
+            for (int q = 0; q < 32; ++q) {  // o = 4q .. 4q+3
+                float sv[4], fv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    sv[u] = Sp[(4 * q + u) * 128 + j];
+                    fv[u] = __bfloat162float(Pt[(4 * q + u) * 128 + j]);
+                }
+                float4 g[8], p[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    g[i] = *reinterpret_cast<const float4*>(smem + RED + red_off(rowi[i], q));
+                    p[i] = *reinterpret_cast<const float4*>(smem + RED + red_off(rowi[i], 32 + q));
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].x, fv[0], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].y, fv[1], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].z, fv[2], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].w, fv[3], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].x, sv[0], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].y, sv[1], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].z, sv[2], acc[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].w, sv[3], acc[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (rc + 2 * i < r1) {
+                    S[(size_t)(rc + 2 * i) * 128 + j] = acc[i];
+                    bad |= !isfinite(acc[i]);
+                }
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, FLAG_NONFINITE);
+    }
+    cluster_sync();  // no CTA leaves while another still reads its shared memory
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+    // when launched as a programmatic dependent of the attention kernel, complete
+    // only after it: later work in the stream stays ordered after both
+    pdl_wait_primary();
 }
 
 }  // namespace tc

@@ -140,7 +140,9 @@ hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc,
                                     float* state, int clean_pass, void* out, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status flags kept
- * in `workspace`: HYB_ERR_TIMEOUT if a bounded device wait gave up,
+ * in `workspace`: HYB_ERR_CUDA if a kernel found its launch environment
+ * unusable (e.g. a misaligned shared-memory window) and did nothing,
+ * else HYB_ERR_TIMEOUT if a bounded device wait gave up,
  * else HYB_WARN_NONFINITE if a state update produced inf/NaN since the last
  * read, else HYB_OK (or HYB_ERR_CUDA if the synchronisation failed). */
 hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
@@ -162,7 +164,8 @@ typedef struct {
 
 hyb_status hyb_attn_timing_begin(int max_launches);
 hyb_status hyb_attn_timing_end(hyb_attn_timing* out);
-/* "prep", "intra_frame_attention", "delta_update_partials", "delta_update_apply"; NULL if out of range */
+/* "prep", "intra_frame_attention", "delta_update" (bf16: the whole update; fp32:
+ * its token-split reduction), "delta_update_apply" (fp32 only); NULL if out of range */
 const char* hyb_attn_kernel_name(int kernel);
 
 /* Static string naming a status code. */
