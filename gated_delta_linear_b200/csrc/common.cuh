@@ -34,10 +34,9 @@ struct LayerArgs {
     // workspace views
     unsigned* flags;
     float* W;                  // fp32 [BH][D][D]: phi_q^T S (SIMT path)
-    __nv_bfloat16* WT_hi;      // bf16 [BH][D][D]: (phi_q^T S)^T, high part (tensor path)
+    __nv_bfloat16* WT_hi;      // bf16 [BH][D][D]: phi_q^T S, row-major, high part (tensor path)
     __nv_bfloat16* WT_lo;      // bf16 [BH][D][D]: low part
-    float* S_prev;             // fp32 [BH][D][D]: copy of S_{N-1} (clean pass)
-    __nv_bfloat16* phivT;      // bf16 [H][D][D]: phi_v transposed (tensor path, clean pass)
+    float* S_prev;             // fp32 [BH][D][D]: copy of S_{N-1} (fp32 path, clean pass)
     float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
     int nsplit;
     int split_tokens;

@@ -62,8 +62,8 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     p->off_W = kStatusBytes;
     p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
     p->off_part = align_up(p->off_Sprev + hh * sizeof(float), 256);
-    // fp32 path: split partials; tensor path: phi_v^T per head
-    const size_t part_bytes = bf16 ? (size_t)d->H * D * D * 2 : hh * 2 * p->nsplit * sizeof(float);
+    // fp32 path: split partials (the tensor path reduces its splits on chip)
+    const size_t part_bytes = bf16 ? 0 : hh * 2 * p->nsplit * sizeof(float);
     p->total = align_up(p->off_part + part_bytes, 256);
     return HYB_OK;
 }
@@ -197,16 +197,33 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
         !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
         !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2))
         return cudaErrorInvalidValue;
-    const dim3 rows(D / simt::kRows, a.H, a.B);
-    e = timed(K_PREP, st, [&] {
-        simt::prep_kernel<D, bf16, true><<<rows, simt::kThreads, prep_smem, st>>>(a, clean);
-    });
+    // Kernels of a pass are chained by programmatic dependent launch: prep waits
+    // for the previous kernel of the stream before it reads the state, then lets
+    // the attention kernel start, which reads prep's W only at its end.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pcfg = {};
+    pcfg.gridDim = dim3(D / simt::kRows, a.H, a.B);
+    pcfg.blockDim = dim3(simt::kThreads, 1, 1);
+    pcfg.dynamicSmemBytes = prep_smem;
+    pcfg.stream = st;
+    pcfg.attrs = pdl;
+    pcfg.numAttrs = 1;
+    cudaError_t le = cudaSuccess;
+    e = timed(K_PREP, st, [&] { le = cudaLaunchKernelEx(&pcfg, simt::prep_kernel<D, bf16, true>, a, clean); });
     if (e != cudaSuccess) return e;
-    const dim3 agrid((a.T + tc::kTile - 1) / tc::kTile, a.H, a.B);
-    e = timed(K_ATTN, st, [&] {
-        tc::attention_kernel<<<agrid, tc::attn::kThreads, tc::attn::SMEM, st>>>(a, tq, tk, tv, tw);
-    });
+    if (le != cudaSuccess) return le;
+    cudaLaunchConfig_t acfg = {};
+    acfg.gridDim = dim3((a.T + tc::kTile - 1) / tc::kTile, a.H, a.B);
+    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::attn::SMEM;
+    acfg.stream = st;
+    acfg.attrs = pdl;
+    acfg.numAttrs = 1;
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw); });
     if (e != cudaSuccess) return e;
+    if (le != cudaSuccess) return le;
     if (clean) {
         // one cluster of nsplit CTAs per (b, h)
         cudaLaunchConfig_t cfg = {};
@@ -225,7 +242,6 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        cudaError_t le = cudaSuccess;
         e = timed(K_UPDATE, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik); });
         if (e != cudaSuccess) return e;
         if (le != cudaSuccess) return le;
@@ -280,7 +296,6 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.WT_lo = a.WT_hi + (size_t)a.B * a.H * p.D * p.D;
     a.S_prev = (float*)(ws + p.off_Sprev);
     a.partials = (float*)(ws + p.off_part);
-    a.phivT = (__nv_bfloat16*)(ws + p.off_part);
     a.nsplit = p.nsplit;
     a.split_tokens = p.split_tokens;
 

@@ -26,9 +26,10 @@ namespace simt {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- prep
-// grid (D/16, H, B): block x computes rows k0..k0+15 of W = phi_q^T S.  S and the
+// grid (D/16, H, B): block x computes rows k0..k0+15 of W = phi_q^T S (row-major;
+// fp32 for the SIMT path, a bf16 hi + lo pair for the tensor path).  S and the
 // block's 16 columns of phi_q are staged in shared memory; each warp owns two
-// rows of W and every lane the columns lane + 32c.
+// rows of W and every lane D/32 consecutive columns.
 constexpr int kRows = 16;
 
 template <int D>
@@ -46,6 +47,13 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
     const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * kRows;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
+    if constexpr (kSplitOut) {
+        // tensor path, launched as a programmatic dependent: wait until the
+        // previous kernel (which may write the state) has completed, then let the
+        // attention kernel start; it reads W only after this grid completes
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     // all loads of a thread are issued before any shared-memory store: the
     // stores go through generic pointers, which would otherwise serialise them
     {
@@ -68,75 +76,49 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
         for (int u = 0; u < NP; ++u) Ph[tid + u * kThreads] = pv[u];
     }
     __syncthreads();
+    // each warp owns rows r0, r0+1 of W; each lane NC consecutive columns
     const int r0 = 2 * warp;
     float acc[2][NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) acc[0][c] = acc[1][c] = 0.f;
 #pragma unroll 4
     for (int o = 0; o < D; ++o) {
-        const float p0 = Ph[o * kRows + r0], p1 = Ph[o * kRows + r0 + 1];
+        const float2 p = *reinterpret_cast<const float2*>(Ph + o * kRows + r0);
+        float sv[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) sv[c] = Ss[o * D + NC * lane + c];
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-            const float sv = Ss[o * D + lane + 32 * c];
-            acc[0][c] = fmaf(p0, sv, acc[0][c]);
-            acc[1][c] = fmaf(p1, sv, acc[1][c]);
+            acc[0][c] = fmaf(p.x, sv[c], acc[0][c]);
+            acc[1][c] = fmaf(p.y, sv[c], acc[1][c]);
         }
     }
-    if (!kSplitOut) {
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr)
+    for (int rr = 0; rr < 2; ++rr) {
+        const size_t row = bh * D * D + (size_t)(k0 + r0 + rr) * D + NC * lane;
+        if constexpr (kSplitOut) {
+            // row-major W as a bf16 hi + lo pair
+            uint32_t hi[NC / 2], lo[NC / 2];
 #pragma unroll
-            for (int c = 0; c < NC; ++c)
-                a.W[bh * D * D + (size_t)(k0 + r0 + rr) * D + lane + 32 * c] = acc[rr][c];
-    } else {
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-            for (int c = 0; c < NC; ++c) Wst[(r0 + rr) * (D + 1) + lane + 32 * c] = acc[rr][c];
-        __syncthreads();
-        // WT[n][k0..k0+15] (K-major B operand of the inter-frame read), hi + lo bf16
-        for (int it = tid; it < 2 * D; it += kThreads) {
-            const int n = it >> 1, half = it & 1;
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float w0 = Wst[(half * 8 + 2 * q) * (D + 1) + n];
-                const float w1 = Wst[(half * 8 + 2 * q + 1) * (D + 1) + n];
-                const __nv_bfloat162 hv = __floats2bfloat162_rn(w0, w1);
-                const __nv_bfloat162 lv = __floats2bfloat162_rn(w0 - __low2float(hv), w1 - __high2float(hv));
-                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
-                lo[q] = *reinterpret_cast<const uint32_t*>(&lv);
+            for (int c = 0; c < NC / 2; ++c) {
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(acc[rr][2 * c], acc[rr][2 * c + 1]);
+                const __nv_bfloat162 lv = __floats2bfloat162_rn(acc[rr][2 * c] - __low2float(hv),
+                                                                acc[rr][2 * c + 1] - __high2float(hv));
+                hi[c] = *reinterpret_cast<const uint32_t*>(&hv);
+                lo[c] = *reinterpret_cast<const uint32_t*>(&lv);
             }
-            const size_t off = bh * D * D + (size_t)n * D + k0 + half * 8;
-            *reinterpret_cast<uint4*>(a.WT_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(a.WT_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint2*>(a.WT_hi + row) = make_uint2(hi[0], hi[1]);
+            *reinterpret_cast<uint2*>(a.WT_lo + row) = make_uint2(lo[0], lo[1]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < NC; ++c) a.W[row + c] = acc[rr][c];
         }
     }
-    if (clean) {
+    if (clean && !kSplitOut) {
+        // the fp32 update reads S_{N-1} from this copy (it writes the state in place)
         float4* dst = reinterpret_cast<float4*>(a.S_prev + bh * D * D + (size_t)k0 * D);
         for (int i = tid; i < kRows * D / 4; i += kThreads)
             dst[i] = reinterpret_cast<const float4*>(Ss + k0 * D)[i];
-    }
-    if constexpr (kSplitOut) {
-        if (clean && b == 0) {
-            // rows k0..k0+15 of phi_v^T (PvT[o][j] = phi_v[j][o]) for the tensor-path update
-            __syncthreads();  // done reading Wst
-            __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(Wst);  // [16][D+8]
-            const __nv_bfloat16* pv = (const __nv_bfloat16*)a.phi_v + (size_t)h * D * D;
-            for (int it = tid; it < 2 * D; it += kThreads) {
-                const int j = it >> 1, half = it & 1;
-                const uint4 v = *reinterpret_cast<const uint4*>(pv + (size_t)j * D + k0 + half * 8);
-                const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) stage[(half * 8 + q) * (D + 8) + j] = e[q];
-            }
-            __syncthreads();
-            for (int it = tid; it < kRows * D / 8; it += kThreads) {
-                const int o = it / (D / 8), c = it % (D / 8);
-                *reinterpret_cast<uint4*>(a.phivT + (size_t)h * D * D + (size_t)(k0 + o) * D + c * 8) =
-                    *reinterpret_cast<const uint4*>(stage + o * (D + 8) + c * 8);
-            }
-        }
     }
 }
 

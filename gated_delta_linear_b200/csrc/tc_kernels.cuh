@@ -12,7 +12,8 @@
 // online softmax from TMEM.  Before the key loop the same Q tile is multiplied
 // by W = phi_q^T S_{N-1} (passed as a two-term bf16 split W_hi + W_lo), so the
 // inter-frame read lands in TMEM next to the softmax accumulator and the
-// epilogue writes out = O_intra + O_inter once.
+// epilogue writes out = O_intra + O_inter once.  W is row-major (rows k), an
+// MN-major B operand.
 //   TMEM columns: [0,128) S (after the key loop: O_inter), [128,256) O,
 //                 [256,320) P buffer 0, [320,384) P buffer 1, [384,448) Q.
 //                 P and Q are bf16, two per 32-bit column, and feed the MMAs
@@ -151,6 +152,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             const int wst = n >= 3 ? (n - 3) % kStages : 2;
             if (ok) ok = mbar_wait(&bars[B_QTMEM], 0, abort_word, a.flags);
             if (ok && n >= 3) ok = mbar_wait(&bars[B_VEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
+            // W comes from the prep kernel, which may still be running when this
+            // grid starts (programmatic dependent launch): wait for it here
+            pdl_wait_primary();
             if (ok) {
                 mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
                 tma_load_3d(sb + Q, &tm_w, &bars[B_W], 0, 0, bh);
@@ -209,10 +213,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tc_fence_after();
                 const int wst = n >= 3 ? (n - 3) % kStages : 2;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tOI, tQ + kk * 8, kmajor_desc(sb + Q, kk), ID_KK, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + Q, kk), ID_KMN, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tOI, tQ + kk * 8, kmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KK, 1);
+                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KMN, 1);
                 mma_commit(&bars[B_OIDONE]);
             }
             // drain: every MMA issued so far completes before TMEM is released
@@ -408,13 +412,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 // ============================================================== delta update
 // One cluster of C CTAs per (batch, head); CTA c of the cluster takes token
 // split c (a run of 128-token tiles) and accumulates its G_c = (beta K')^T K'
-// and P_c = (beta K')^T V in TMEM.  The CTAs then park [G_c | P_c] in shared
-// memory, each reduces its own band of rows over the C CTAs through
-// distributed shared memory (fixed order c = 0..C-1, so the result is
-// deterministic), and applies the update to that band:
-//   S_N[i][:] = alpha S_{N-1}[i][:] + P[i][:] phi_v^T - G[i][:] S_{N-1}
-// with alpha = mean_t sigmoid(g_t); S_{N-1} and phi_v^T come from the
-// workspace (written by the prep kernel of the same pass).
+// and P_c = (beta K')^T V in TMEM.  Since the update is linear in the splits,
+// every CTA then forms its own contribution Delta_c = P_c phi_v^T - G_c S_{N-1}
+// on the tensor core (bf16 hi + lo splits of G_c, P_c and S_{N-1}), and each
+// CTA sums one band of rows of Delta over the C CTAs through distributed
+// shared memory (fixed order c = 0..C-1, so the result is deterministic):
+//   S_N[i][:] = alpha S_{N-1}[i][:] + sum_c Delta_c[i][:]
+// with alpha = mean_t sigmoid(g_t).  Every CTA stages S_{N-1} from the state
+// buffer before the cluster's first barrier and writes its band after it.  The
+// kernel reads only the pass's inputs and the state, never the prep kernel's
+// outputs, so it may run alongside the attention kernel.
 namespace upd {
 // tile loop (1024-aligned 128B-swizzled tiles)
 constexpr uint32_t PHI = 0;
@@ -426,20 +433,22 @@ constexpr uint32_t KH = AL + kTileBytes;
 constexpr uint32_t KL = KH + kTileBytes;
 constexpr uint32_t TILES_END = KL + kTileBytes;          // 229,376
 // after the tile loop (reuses the tile space)
-constexpr uint32_t PHIVT = 0;                             // phi_v^T bf16 [128][128]
-constexpr uint32_t SPREV = PHIVT + 128 * 128 * 2;         // S_{N-1} fp32 [128][128]
-constexpr uint32_t RED = SPREV + 128 * 128 * 4;           // [128][256] fp32, 16-byte chunks XOR-swizzled by row
+constexpr uint32_t PHIV = 0;                              // phi_v, K-major B operand (rows j, o contiguous)
+constexpr uint32_t SPREV = PHIV + kTileBytes;             // S_{N-1} fp32 [128][128]
+constexpr uint32_t SH = SPREV + 128 * 128 * 4;            // S_hi, MN-major B operand (rows m, j contiguous)
+constexpr uint32_t SL = SH + kTileBytes;                  // S_lo
+constexpr uint32_t RED = SL + kTileBytes;                 // Delta_c fp32 [128][128], 16-byte chunks XOR-swizzled
 constexpr uint32_t BAR = TILES_END;                       // barriers, TMEM slot, flags, sums
 constexpr uint32_t XSS = BAR + 256;                       // [2 parity][2 halves][128 rows] floats + ok bytes
 constexpr uint32_t SMEM = XSS + 2048 + 512;               // 232,192 B
 constexpr int kNormThreads = 256;                         // warps 0-7
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
-enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_OPSFULL, B_OPSFREE, B_PARK, B_COUNT };
-static_assert(RED + 128 * 256 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
-// byte offset of float4 chunk q (0..63) of row `row` in RED
+enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_OPSFULL, B_OPSFREE, B_PARK, B_DELTA, B_COUNT };
+static_assert(RED + 128 * 128 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
+// byte offset of float4 chunk q (0..31) of row `row` in RED
 __device__ __forceinline__ uint32_t red_off(int row, int q) {
-    return (uint32_t)(row * 1024 + ((q ^ (row & 7)) << 4));
+    return (uint32_t)(row * 512 + ((q ^ (row & 7)) << 4));
 }
 }  // namespace upd
 
@@ -630,14 +639,17 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         if (ok && nt > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OPSFREE], (nt - 1) & 1, abort_word, a.flags));
     }
-    // ------------------------------------------------------------ park [G | P]; stage S_{N-1}, phi_v^T
+    // ------------------------------------------------------------ Delta_c = P_c phi_v^T - G_c S_{N-1}
+    // G_c and P_c (fp32 in TMEM) become bf16 hi + lo A operands in TMEM; S_{N-1}
+    // becomes a bf16 hi + lo B operand and phi_v a K-major B operand in shared
+    // memory; five MMAs give this split's contribution, which the cluster sums.
+    const uint32_t tGH = tmem, tGL = tmem + 64, tD = tmem + 128, tPH = tmem + 384, tPL = tmem + 448;
     tc_fence_before();
-    __syncthreads();  // every MMA has completed (or timed out): the tile space is free
+    __syncthreads();  // every MMA of the tile loop has completed (or timed out)
     tc_fence_after();
     if (threadIdx.x == kLoadWarp * 32) {
-        mbar_expect_tx(&bars[B_PARK], 128 * 128 * 2 + 128 * 128 * 4);
-        bulk_load(sb + PHIVT, a.phivT + (size_t)h * 128 * 128, 128 * 128 * 2, &bars[B_PARK]);
-        bulk_load(sb + SPREV, a.S_prev + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
+        mbar_expect_tx(&bars[B_PARK], 128 * 128 * 4);
+        bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
     }
     {
         float sg = 0.f;
@@ -646,26 +658,107 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         for (int o = 16; o > 0; o >>= 1) sg += __shfl_xor_sync(0xffffffffu, sg, o);
         if (lane == 0) wsum[warp] = sg;
     }
+    bool park_ok = true;
     if (warp < 8) {
-        // this warp's rows, columns [64 half, 64 half + 64) of G and of P
         const int half = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        // phi_v row `row`, columns 64 half..+63, into the K-major B tile
+        {
+            const uint4* src = reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.phi_v +
+                                                              (size_t)h * 128 * 128 + (size_t)row * 128 + half * 64);
+            uint4 v[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) v[c] = src[c];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(smem + PHIV + half * kHalf + sw128_offset(row, c)) = v[c];
+        }
+        // G and P rows `row`, columns 64 half..+63: fp32 -> bf16 hi + lo in TMEM
+#pragma unroll
+        for (int gp = 0; gp < 2; ++gp) {
+            float x[64];
+            uint32_t hi[32], lo[32];
+            const uint32_t src = (gp == 0 ? tG : tP) + lrow + half * 64;
+            if (nt > 0) {
+                tmem_ld32(src, x);
+                tmem_ld32(src + 32, x + 32);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int q = 0; q < 64; ++q) x[q] = 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
+                lo[q] = pack_bf16(x[2 * q] - __low2float(hv), x[2 * q + 1] - __high2float(hv));
+            }
+            tmem_st32u((gp == 0 ? tGH : tPH) + lrow + half * 32, hi);
+            tmem_st32u((gp == 0 ? tGL : tPL) + lrow + half * 32, lo);
+        }
+        tmem_st_wait();
+        // S_{N-1} row `row`, columns 64 half..+63: bf16 hi + lo into the MN-major B tiles
+        park_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PARK], 0, abort_word, a.flags));
+        const float* Sp = reinterpret_cast<const float*>(smem + SPREV) + row * 128 + half * 64;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float s0 = Sp[8 * c + 2 * q], s1 = Sp[8 * c + 2 * q + 1];
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(s0, s1);
+                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
+                lo[q] = pack_bf16(s0 - __low2float(hv), s1 - __high2float(hv));
+            }
+            const uint32_t off = half * kHalf + sw128_offset(row, c);
+            *reinterpret_cast<uint4*>(smem + SH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(smem + SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    } else {
+        // S_{N-1} must be in shared memory before any CTA of the cluster passes the
+        // first cluster barrier: after it, CTAs write their bands of the state
+        park_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PARK], 0, abort_word, a.flags));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == kMmaWarp * 32) {
+        constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t ID_KMN_NEG = idesc_bf16(128, 128, 0, 1) | (1u << 13);  // -A
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tD, tPH + kk * 8, kmajor_desc(sb + PHIV, kk), ID_KK, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tD, tPL + kk * 8, kmajor_desc(sb + PHIV, kk), ID_KK, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tD, tGH + kk * 8, mnmajor_desc(sb + SH, kk), ID_KMN_NEG, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tD, tGH + kk * 8, mnmajor_desc(sb + SL, kk), ID_KMN_NEG, 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tD, tGL + kk * 8, mnmajor_desc(sb + SH, kk), ID_KMN_NEG, 1);
+        mma_commit(&bars[B_DELTA]);
+    }
+    if (warp < 8) {
+        // Delta_c row `row`, columns 64 half..+63, into shared memory for the cluster
+        const int half = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        const bool d_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_DELTA], 0, abort_word, a.flags));
+        tc_fence_after();
         float v[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // c: G lo, G hi, P lo, P hi (32 columns each)
-            const uint32_t src = (c < 2 ? tG : tP) + lrow + half * 64 + (c & 1) * 32;
-            if (nt > 0) {
-                tmem_ld32(src, v);
+        for (int c = 0; c < 2; ++c) {
+            if (d_ok) {
+                tmem_ld32(tD + lrow + half * 64 + c * 32, v);
                 tmem_ld_wait();
             } else {
 #pragma unroll
                 for (int q = 0; q < 32; ++q) v[q] = 0.f;
             }
-            const int q0 = (c >> 1) * 32 + half * 16 + (c & 1) * 8;  // first float4 chunk
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4*>(smem + RED + red_off(row, q0 + q)) =
+                *reinterpret_cast<float4*>(smem + RED + red_off(row, half * 16 + c * 8 + q)) =
                     make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
     }
@@ -675,19 +768,24 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         for (int w = 0; w < kThreads / 32; ++w) t += wsum[w];
         wsum[10] = t / (float)T;
     }
-    cluster_sync();  // every CTA of the cluster has parked its [G | P]
+    cluster_sync();  // every CTA of the cluster has parked Delta_c and staged S_{N-1}
 
-    // ------------------------------------------------------------ reduce this CTA's band of rows
-    const int band = (128 + C - 1) / C;
-    const int r0 = min(128, split * band), r1 = min(128, r0 + band);
+    // ------------------------------------------------------------ reduce and apply this CTA's band
+    // S_N[row] = alpha S_{N-1}[row] + sum_c Delta_c[row], ranks summed in order
     {
-        const int items = (r1 - r0) * 64;
-        // two items per step, all their C remote loads in flight together
-        for (int it = threadIdx.x; it < items; it += 2 * kThreads) {
+        const int band = (128 + C - 1) / C;
+        const int r0 = min(128, split * band), r1 = min(128, r0 + band);
+        const float alpha = wsum[10];
+        const float* Sp = reinterpret_cast<const float*>(smem + SPREV);
+        float* S = a.state + (size_t)bh * 128 * 128;
+        const int items = (r1 - r0) * 32;
+        bool bad = false;
+        for (int it = threadIdx.x; it < items && park_ok; it += 2 * kThreads) {
             const int it2 = it + kThreads;
             const bool second = it2 < items;
-            const uint32_t off0 = red_off(r0 + it / 64, it % 64);
-            const uint32_t off1 = second ? red_off(r0 + it2 / 64, it2 % 64) : off0;
+            const int row0 = r0 + it / 32, q0 = it % 32;
+            const int row1 = second ? r0 + it2 / 32 : row0, q1 = second ? it2 % 32 : q0;
+            const uint32_t off0 = red_off(row0, q0), off1 = red_off(row1, q1);
             float4 v0[kMaxClusterRanks], v1[kMaxClusterRanks];
 #pragma unroll
             for (int c = 0; c < kMaxClusterRanks; ++c)
@@ -695,75 +793,22 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
                     v0[c] = ld_cluster_f4(sb + RED + off0, (uint32_t)c);
                     v1[c] = ld_cluster_f4(sb + RED + off1, (uint32_t)c);
                 }
-            float4 s0 = v0[0], s1 = v1[0];
+            float4 s0 = *reinterpret_cast<const float4*>(Sp + row0 * 128 + q0 * 4);
+            float4 s1 = *reinterpret_cast<const float4*>(Sp + row1 * 128 + q1 * 4);
+            s0 = make_float4(alpha * s0.x, alpha * s0.y, alpha * s0.z, alpha * s0.w);
+            s1 = make_float4(alpha * s1.x, alpha * s1.y, alpha * s1.z, alpha * s1.w);
 #pragma unroll
-            for (int c = 1; c < kMaxClusterRanks; ++c)
+            for (int c = 0; c < kMaxClusterRanks; ++c)
                 if (c < C) {
                     s0.x += v0[c].x; s0.y += v0[c].y; s0.z += v0[c].z; s0.w += v0[c].w;
                     s1.x += v1[c].x; s1.y += v1[c].y; s1.z += v1[c].z; s1.w += v1[c].w;
                 }
-            *reinterpret_cast<float4*>(smem + RED + off0) = s0;
-            if (second) *reinterpret_cast<float4*>(smem + RED + off1) = s1;
-        }
-    }
-    const bool park_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PARK], 0, abort_word, a.flags));
-    __syncthreads();
-
-    // ------------------------------------------------------------ apply to the band
-    if (warp < 8 && park_ok) {
-        const int j = threadIdx.x & 127;  // output column
-        const int rs = threadIdx.x >> 7;  // this thread takes rows r0 + rs, r0 + rs + 2, ...
-        const float alpha = wsum[10];
-        const float* Sp = reinterpret_cast<const float*>(smem + SPREV);
-        const __nv_bfloat16* Pt = reinterpret_cast<const __nv_bfloat16*>(smem + PHIVT);
-        float* S = a.state + (size_t)bh * 128 * 128;
-        bool bad = false;
-        for (int rc = r0 + rs; rc < r1; rc += 16) {
-            // rows rc, rc + 2, ..., rc + 14; rows at or past r1 are computed on
-            // clamped (valid) data and discarded
-            int rowi[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) rowi[i] = min(rc + 2 * i, 127);
-            float acc[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = alpha * Sp[rowi[i] * 128 + j];
-#pragma unroll 2
-            for (int q = 0; q < 32; ++q) {  // o = 4q .. 4q+3
-                float sv[4], fv[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    sv[u] = Sp[(4 * q + u) * 128 + j];
-                    fv[u] = __bfloat162float(Pt[(4 * q + u) * 128 + j]);
-                }
-                float4 g[8], p[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    g[i] = *reinterpret_cast<const float4*>(smem + RED + red_off(rowi[i], q));
-                    p[i] = *reinterpret_cast<const float4*>(smem + RED + red_off(rowi[i], 32 + q));
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].x, fv[0], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].y, fv[1], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].z, fv[2], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(p[i].w, fv[3], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].x, sv[0], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].y, sv[1], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].z, sv[2], acc[i]);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(-g[i].w, sv[3], acc[i]);
+            *reinterpret_cast<float4*>(S + row0 * 128 + q0 * 4) = s0;
+            bad |= !(isfinite(s0.x) && isfinite(s0.y) && isfinite(s0.z) && isfinite(s0.w));
+            if (second) {
+                *reinterpret_cast<float4*>(S + row1 * 128 + q1 * 4) = s1;
+                bad |= !(isfinite(s1.x) && isfinite(s1.y) && isfinite(s1.z) && isfinite(s1.w));
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (rc + 2 * i < r1) {
-                    S[(size_t)(rc + 2 * i) * 128 + j] = acc[i];
-                    bad |= !isfinite(acc[i]);
-                }
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, FLAG_NONFINITE);
     }
