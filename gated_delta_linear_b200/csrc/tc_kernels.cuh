@@ -14,17 +14,16 @@
 // inter-frame read lands in TMEM next to the softmax accumulator and the
 // epilogue writes out = O_intra + O_inter once.  W is row-major (rows k), an
 // MN-major B operand.
-//   TMEM columns: [0,128) S (after the key loop: O_inter), [128,256) O,
-//                 [256,320) P buffer 0, [320,384) P buffer 1, [384,448) Q.
-//                 P and Q are bf16, two per 32-bit column, and feed the MMAs
-//                 as A operands, so per key tile shared memory only carries K
-//                 and V.  As soon as both softmax halves have read S_j, the MMA
-//                 warp issues S_{j+1} into the same columns, so the next tile's
-//                 scores are computed while the softmax exponentiates this one.
-//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Q moves to TMEM at
-//                 the start; W_hi then takes its buffer and W_lo a V stage the
-//                 key loop no longer needs, and O_inter = Q W_hi + Q W_lo is
-//                 computed while the softmax works on the last tile.
+//   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
+//                 [384,448) P buffer 0, [448,512) P buffer 1 (bf16, two per
+//                 32-bit column, the A operand of P.V).  As soon as both
+//                 softmax halves have read S_j, the MMA warp issues S_{j+2}
+//                 into its buffer, ahead of P_j.V_j, so the scores of a tile
+//                 are always ready before the softmax reaches it.
+//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  At the end W_hi and
+//                 W_lo take the K and V stages of tile n-3 (unused stage 2 when
+//                 n < 3) and O_inter = Q W_hi + Q W_lo goes to the S buffer
+//                 the last tile does not use, while the softmax finishes.
 //   Every CTA signals at entry that the next kernel (the delta update, which
 //   reads none of this kernel's outputs) may start on idle SMs.
 //
@@ -63,8 +62,8 @@ constexpr uint32_t SMEM = XOK + 512;          // 232,192 B
 constexpr int kSoftmaxThreads = 256;           // warps 0-7
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
-enum { B_Q = 0, B_QTMEM = 1, B_W = 2, B_OIDONE = 3, B_KFULL = 4, B_KEMPTY = 7, B_VFULL = 10,
-       B_VEMPTY = 13, B_SFULL = 16, B_SREAD = 17, B_PFULL = 18, B_PVDONE = 20, B_COUNT = 22 };
+enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12,
+       B_SFULL = 15, B_SREAD = 17, B_PFULL = 19, B_PVDONE = 21, B_COUNT = 23 };
 }  // namespace attn
 
 // K-major operand, 128 rows x 128 bf16 stored as two 64-column swizzled boxes:
@@ -108,7 +107,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1 || i == B_SREAD || i == B_QTMEM)
+            mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1 || i == B_SREAD || i == B_SREAD + 1)
                                     ? kSoftmaxThreads
                                     : 1);
         *abort_word = 0;
@@ -119,8 +118,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128, tP0 = tmem + 256, tQ = tmem + 384;
-    const uint32_t tOI = tS;  // O_inter reuses the S columns after the last softmax read
+    const uint32_t tS0 = tmem, tO = tmem + 256, tP0 = tmem + 384;
+    const uint32_t tOI = tS0 + (n & 1) * 128;  // the S buffer the last tile does not use
 
     if (warp == kLoadWarp) {
         // ------------------------------------------------ TMA producer
@@ -146,19 +145,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tma_load_3d(sb + V0 + st * kTileBytes, &tm_v, &bars[B_VFULL + st], xh, j * kTile, b);
                 tma_load_3d(sb + V0 + st * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + st], xh + 64, j * kTile, b);
             }
-            // W_hi into the Q buffer once Q is in TMEM; W_lo into the V stage of
-            // tile n-3 once PV_{n-3} has read it (stage 2, never used, when n < 3)
+            // W_hi / W_lo into the K / V stages of tile n-3 once S_{n-3} / PV_{n-3}
+            // have read them (stage 2, never used, when n < 3)
             const int nbh = a.B * a.H;
             const int wst = n >= 3 ? (n - 3) % kStages : 2;
-            if (ok) ok = mbar_wait(&bars[B_QTMEM], 0, abort_word, a.flags);
+            if (ok && n >= 3) ok = mbar_wait(&bars[B_KEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
             if (ok && n >= 3) ok = mbar_wait(&bars[B_VEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
             // W comes from the prep kernel, which may still be running when this
             // grid starts (programmatic dependent launch): wait for it here
             pdl_wait_primary();
             if (ok) {
                 mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
-                tma_load_3d(sb + Q, &tm_w, &bars[B_W], 0, 0, bh);
-                tma_load_3d(sb + Q + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
+                tma_load_3d(sb + K0 + wst * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
+                tma_load_3d(sb + K0 + wst * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
                 tma_load_3d(sb + V0 + wst * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
                 tma_load_3d(sb + V0 + wst * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
             }
@@ -169,30 +168,32 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            bool ok = mbar_wait(&bars[B_QTMEM], 0, abort_word, a.flags);
-            if (ok) {
-                ok = mbar_wait(&bars[B_KFULL], 0, abort_word, a.flags);
-                if (ok) {
-                    tc_fence_after();
+            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags);
+            for (int j = 0; j < 2 && j < n && ok; ++j) {
+                ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tS, tQ + kk * 8, kmajor_desc(sb + K0, kk), ID_KK, kk > 0);
-                    mma_commit(&bars[B_SFULL]);
-                    mma_commit(&bars[B_KEMPTY]);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK,
+                             kk > 0);
+                mma_commit(&bars[B_SFULL + j]);
+                mma_commit(&bars[B_KEMPTY + j]);
             }
             for (int j = 0; j < n && ok; ++j) {
-                if (j + 1 < n) {
-                    // S_{j+1} into the S columns once both halves have read S_j
-                    const int st1 = (j + 1) % kStages;
-                    if (!mbar_wait(&bars[B_SREAD], j & 1, abort_word, a.flags)) break;
-                    if (!mbar_wait(&bars[B_KFULL + st1], ((j + 1) / kStages) & 1, abort_word, a.flags)) break;
+                const int sb2 = j & 1;
+                if (j + 2 < n) {
+                    // S_{j+2} into S buffer j&1 once both halves have read S_j
+                    const int st2 = (j + 2) % kStages;
+                    if (!mbar_wait(&bars[B_SREAD + sb2], (j >> 1) & 1, abort_word, a.flags)) break;
+                    if (!mbar_wait(&bars[B_KFULL + st2], ((j + 2) / kStages) & 1, abort_word, a.flags)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tS, tQ + kk * 8, kmajor_desc(sb + K0 + st1 * kTileBytes, kk), ID_KK, kk > 0);
-                    mma_commit(&bars[B_SFULL]);
-                    mma_commit(&bars[B_KEMPTY + st1]);
+                        mma_bf16(tS0 + sb2 * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + st2 * kTileBytes, kk),
+                                 ID_KK, kk > 0);
+                    mma_commit(&bars[B_SFULL + sb2]);
+                    mma_commit(&bars[B_KEMPTY + st2]);
                 }
                 const int pb = j & 1, st = j % kStages;
                 if (!mbar_wait(&bars[B_PFULL + pb], (j >> 1) & 1, abort_word, a.flags)) break;
@@ -206,17 +207,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 mma_commit(&bars[B_PVDONE + pb]);
                 mma_commit(&bars[B_VEMPTY + st]);
             }
-            // O_inter = Q W_hi + Q W_lo into the S columns, once the last S is read
-            if (ok) ok = mbar_wait(&bars[B_SREAD], (n - 1) & 1, abort_word, a.flags);
+            // O_inter = Q W_hi + Q W_lo into S buffer n&1, once S_{n-2} has been read
+            if (ok && n >= 2) ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags);
             if (ok) ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags);
             if (ok) {
                 tc_fence_after();
                 const int wst = n >= 3 ? (n - 3) % kStages : 2;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + Q, kk), ID_KMN, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), mnmajor_desc(sb + K0 + wst * kTileBytes, kk), ID_KMN,
+                             kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KMN, 1);
+                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), mnmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KMN, 1);
                 mma_commit(&bars[B_OIDONE]);
             }
             // drain: every MMA issued so far completes before TMEM is released
@@ -239,39 +242,23 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
         const float scale = a.sm_scale_log2;
         float m = -INFINITY, l = 0.f;
-        // Q row r, features 64ch..64ch+63, from the swizzled TMA tile into TMEM
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags));
-        if (ok) {
-            uint32_t qv[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + ch * kHalf + sw128_offset(r, c));
-                qv[4 * c + 0] = v.x;
-                qv[4 * c + 1] = v.y;
-                qv[4 * c + 2] = v.z;
-                qv[4 * c + 3] = v.w;
-            }
-            tmem_st32u(tQ + lrow + ch * 32, qv);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[B_QTMEM]);
-        }
+        bool ok = true;
         float x[64];
         for (int j = 0; j < n; ++j) {
             const int s = j & 1;
             // waits of this iteration: S_j ready; P buffer s free (PV_{j-2} done)
-            bool w_ok = ok && mbar_wait(&bars[B_SFULL], j & 1, abort_word, a.flags);
+            bool w_ok = ok && mbar_wait(&bars[B_SFULL + s], (j >> 1) & 1, abort_word, a.flags);
             if (j >= 2) w_ok = w_ok && mbar_wait(&bars[B_PVDONE + s], ((j >> 1) + 1) & 1, abort_word, a.flags);
             w_ok = __all_sync(0xffffffffu, w_ok);
             float hm = -INFINITY;
             if (w_ok) {
                 tc_fence_after();
-                tmem_ld32(tS + lrow + ch * 64, x);
-                tmem_ld32(tS + lrow + ch * 64 + 32, x + 32);
+                tmem_ld32(tS0 + s * 128 + lrow + ch * 64, x);
+                tmem_ld32(tS0 + s * 128 + lrow + ch * 64 + 32, x + 32);
                 tmem_ld_wait();
-                // S_j is in registers: the MMA warp may overwrite it with S_{j+1}
+                // S_j is in registers: the MMA warp may overwrite it with S_{j+2}
                 tc_fence_before();
-                mbar_arrive(&bars[B_SREAD]);
+                mbar_arrive(&bars[B_SREAD + s]);
                 const int valid = T - j * kTile - ch * 64;
                 if (valid < 64) {
 #pragma unroll
