@@ -109,6 +109,11 @@ cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     if (done[dev]) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    // every kernel of a pass asks for the same (largest) shared-memory carveout, so
+    // an SM freed by one kernel takes the next one's CTAs without reconfiguring
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) done[dev] = 1;
     return e;
 }

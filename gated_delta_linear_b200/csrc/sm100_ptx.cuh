@@ -234,28 +234,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for x <= 8: Cody-Waite range reduction x = n + f,
-// n = round(x) (found by adding 1.5 * 2^23), f in [-1/2, 1/2]; 2^f from a
-// degree-3 minimax polynomial (Remez, relative error 7.5e-5 on the interval;
-// coefficients from gen_exp2_poly.py); 2^n added to the exponent field.
-// x is clamped to -125 so the result stays a normal float (about 2.4e-38 at
-// the clamp, where the exact value would be smaller).
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999280571937561f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two non-negative floats to a bf16 pair (lo in the low half) on the integer
-// pipe: round half up at bit 16, then keep the high halves.
-__device__ __forceinline__ uint32_t pack_bf16_rhu(float lo, float hi) {
-    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

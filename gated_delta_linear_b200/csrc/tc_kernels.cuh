@@ -6,24 +6,28 @@
 // inter-frame read O_inter = Q' S_{N-1}, gated delta update) and §2.2
 // (frame-level access: all tokens read the pre-update state).
 //
-// intra_frame_attention: one CTA per (128-query tile, head, batch).  Warp 4
-// streams Q, K and V tiles with TMA into 128B-swizzled shared memory; warp 5
-// issues the tcgen05 MMAs; warps 0-3 own one query row per thread and run the
-// online softmax from TMEM.  Before the key loop the same Q tile is multiplied
-// by W = phi_q^T S_{N-1} (passed as a two-term bf16 split W_hi + W_lo), so the
-// inter-frame read lands in TMEM next to the softmax accumulator and the
-// epilogue writes out = O_intra + O_inter once.  W is row-major (rows k), an
-// MN-major B operand.
+// intra_frame_attention: one CTA per (128-query tile, head, batch), 7 warps.
+// Warp 4 streams Q and the K ring, warp 6 the V ring, with TMA into
+// 128B-swizzled shared memory; warp 5 issues the tcgen05 MMAs; warps 0-3 own
+// one query row per thread (a TMEM lane) and run the online softmax with all
+// 128 scores of a key tile in registers.  After the key loop the Q tile is
+// multiplied by W = phi_q^T S_{N-1} (a two-term bf16 split W_hi + W_lo, row
+// major: an MN-major B operand), so the inter-frame read lands in TMEM next to
+// the softmax accumulator and the epilogue writes out = O_intra + O_inter once.
 //   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
-//                 [384,448) P buffer 0, [448,512) P buffer 1 (bf16, two per
-//                 32-bit column, the A operand of P.V).  As soon as both
-//                 softmax halves have read S_j, the MMA warp issues S_{j+2}
-//                 into its buffer, ahead of P_j.V_j, so the scores of a tile
-//                 are always ready before the softmax reaches it.
+//                 [384,448) Q, [448,512) P (bf16, two per 32-bit column: the
+//                 A operands of S = Q K^T and O += P V).  Q is copied from
+//                 shared memory into TMEM once; as soon as the softmax has S_j
+//                 in registers the MMA warp issues S_{j+2} into its buffer, so
+//                 scores run a tile ahead of the softmax, and the softmax loads
+//                 S_{j+1} while it hands P_j over.
+//   Softmax: exponents against a running offset (the first tile's row max),
+//                 moved only when a tile's partial sum leaves [0, 2^64); all
+//                 exponentials on the MUFU pipe.
 //   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  At the end W_hi and
-//                 W_lo take the K and V stages of tile n-3 (unused stage 2 when
-//                 n < 3) and O_inter = Q W_hi + Q W_lo goes to the S buffer
-//                 the last tile does not use, while the softmax finishes.
+//                 W_lo take the K stages of key tiles n-3 and n-2 (unused
+//                 stages when n < 3) and O_inter = Q W_hi + Q W_lo goes to the
+//                 S buffer the last tile does not use.
 //   Every CTA signals at entry that the next kernel (the delta update, which
 //   reads none of this kernel's outputs) may start on idle SMs.
 //
@@ -51,19 +55,19 @@ constexpr int kMaxClusterRanks = 8;             // token splits per (b, h) in th
 
 // ============================================================== attention
 namespace attn {
-constexpr int kStages = 3;                     // K and V ring depth
+constexpr int kKStages = 3;                    // K ring depth
+constexpr int kVStages = 3;                    // V ring depth
 constexpr uint32_t Q = 0;
 constexpr uint32_t K0 = Q + kTileBytes;
-constexpr uint32_t V0 = K0 + kStages * kTileBytes;
-constexpr uint32_t BAR = V0 + kStages * kTileBytes;
-constexpr uint32_t XCHG = BAR + 256;          // softmax pair exchange: [2][2][128] floats
-constexpr uint32_t XOK = XCHG + 2048;         // and [2][2][128] wait results (bytes)
-constexpr uint32_t SMEM = XOK + 512;          // 232,192 B
-constexpr int kSoftmaxThreads = 256;           // warps 0-7
-constexpr int kLoadWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
-enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12,
-       B_SFULL = 15, B_SREAD = 17, B_PFULL = 19, B_PVDONE = 21, B_COUNT = 23 };
+constexpr uint32_t V0 = K0 + kKStages * kTileBytes;
+constexpr uint32_t BAR = V0 + kVStages * kTileBytes;
+constexpr uint32_t SMEM = BAR + 256;           // 229,632 B
+constexpr int kSoftmaxThreads = 128;           // warps 0-3, one query row per thread
+constexpr int kLoadWarp = 4, kMmaWarp = 5, kLoadVWarp = 6;
+constexpr int kThreads = 224;
+enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12, B_SFULL = 15,
+       B_SREAD = 17, B_QTM = 19, B_PFULL = 20, B_PVDONE = 21, B_COUNT = 22 };
+static_assert(B_COUNT * 8 + 8 <= 256, "barrier block");
 }  // namespace attn
 
 // K-major operand, 128 rows x 128 bf16 stored as two 64-column swizzled boxes:
@@ -74,6 +78,35 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
 // MN-major operand with the same storage (rows = K index): slice kk covers K rows 16kk..16kk+15.
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     return sdesc_sw128(base + kk * 2048, kHalf, 1024);
+}
+
+// Row max of 128 scores (fmaxf: NaN entries are skipped).
+__device__ __forceinline__ float row_max128(const float* x) {
+    float m8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        m8[k] = fmaxf(fmaxf(x[k], x[k + 8]), fmaxf(x[k + 16], x[k + 24]));
+#pragma unroll
+        for (int c = 32; c < 128; c += 32)
+            m8[k] = fmaxf(m8[k], fmaxf(fmaxf(x[c + k], x[c + k + 8]), fmaxf(x[c + k + 16], x[c + k + 24])));
+    }
+    return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
+// p = 2^(x * scale + neg_m) for one row's 128 scores, as 64 bf16 pairs (round
+// to nearest) in pk; returns the row sum of p in fp32 (the exponentials on the
+// MUFU pipe, the pair conversion one instruction per two values).
+__device__ __forceinline__ float exp_tile(const float* x, float scale, float neg_m, uint32_t* pk) {
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 64; ++k) {
+        const float e0 = ex2(fmaf(x[2 * k], scale, neg_m));
+        const float e1 = ex2(fmaf(x[2 * k + 1], scale, neg_m));
+        l4[(2 * k) & 3] += e0;
+        l4[(2 * k + 1) & 3] += e1;
+        pk[k] = pack_bf16(e0, e1);
+    }
+    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
 __global__ void __launch_bounds__(attn::kThreads, 1)
@@ -88,138 +121,155 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
         return;
     }
+    // the delta update of this pass does not read anything this kernel writes:
+    // it may start on SMs this grid leaves idle
+    pdl_launch_dependents();
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
     volatile int* abort_word = (volatile int*)(tmem_slot + 1);
-    float* xchg = (float*)(smem + XCHG);    // [2 parity][2 halves][128 rows] row maxima, then row sums
-    uint8_t* xok = smem + XOK;              // [2 parity][2 halves][128 rows] wait results
 
-    // the delta update of this pass does not read anything this kernel writes:
-    // it may start on SMs this grid leaves idle
-    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T;
-    const int q0 = qt * kTile;
+    const int q0 = qt_ * kTile;
     const int n = (T + kTile - 1) / kTile;
     const int bh = b * a.H + h;
+    // K stages that receive W_hi / W_lo at the end (free once the scores of key
+    // tiles n-3 / n-2 are computed; stages no tile uses when n is small)
+    const int wst_hi = n >= 3 ? (n - 3) % kKStages : 2;
+    const int wst_lo = n >= 2 ? (n - 2) % kKStages : 1;
 
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == kLoadWarp * 32) {
+        // the producer initialises the barriers and starts the first loads
+        // before the block synchronises (the loads land on its own barriers)
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1 || i == B_SREAD || i == B_SREAD + 1)
-                                    ? kSoftmaxThreads
-                                    : 1);
+            mbar_init(&bars[i],
+                      (i == B_PFULL || i == B_QTM || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads : 1);
         *abort_word = 0;
         fence_mbar_init();
+        fence_async_smem();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        const int xh = h * 128;
+        mbar_expect_tx(&bars[B_Q], kTileBytes);
+        tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0, b);
+        tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
+        for (int j = 0; j < kKStages && j < n; ++j) {
+            mbar_expect_tx(&bars[B_KFULL + j], kTileBytes);
+            tma_load_3d(sb + K0 + j * kTileBytes, &tm_k, &bars[B_KFULL + j], xh, j * kTile, b);
+            tma_load_3d(sb + K0 + j * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + j], xh + 64, j * kTile, b);
+        }
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tO = tmem + 256, tP0 = tmem + 384;
+    // S buffers 0 / 1, O, Q and P as bf16 pairs (the A operands of the score
+    // and value products)
+    const uint32_t tS0 = tmem, tO = tmem + 256, tQ = tmem + 384, tP = tmem + 448;
     const uint32_t tOI = tS0 + (n & 1) * 128;  // the S buffer the last tile does not use
 
-    if (warp == kLoadWarp) {
-        // ------------------------------------------------ TMA producer
+    if (warp == kLoadVWarp) {
+        // ------------------------------------------------ TMA producer: V ring
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            const int xh = h * 128;
+            for (int j = 0; j < n; ++j) {
+                const int vs = j % kVStages;
+                if (j >= kVStages &&
+                    !mbar_wait(&bars[B_VEMPTY + vs], ((j / kVStages) + 1) & 1, abort_word, a.flags))
+                    break;
+                mbar_expect_tx(&bars[B_VFULL + vs], kTileBytes);
+                tma_load_3d(sb + V0 + vs * kTileBytes, &tm_v, &bars[B_VFULL + vs], xh, j * kTile, b);
+                tma_load_3d(sb + V0 + vs * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + vs], xh + 64, j * kTile, b);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kLoadWarp) {
+        // ------------------------------------------------ TMA producer: Q, K ring, W
+        // (its own warp, so K tiles run ahead of the V ring's waits)
+        if (lane == 0) {
             tma_prefetch_desc(&tm_w);
             const int xh = h * 128;
-            mbar_expect_tx(&bars[B_Q], kTileBytes);
-            tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0, b);
-            tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
             bool ok = true;
-            for (int j = 0; j < n && ok; ++j) {
-                const int st = j % kStages;
-                const uint32_t par = ((j / kStages) + 1) & 1;
-                if (j >= kStages && !(ok = mbar_wait(&bars[B_KEMPTY + st], par, abort_word, a.flags))) break;
-                mbar_expect_tx(&bars[B_KFULL + st], kTileBytes);
-                tma_load_3d(sb + K0 + st * kTileBytes, &tm_k, &bars[B_KFULL + st], xh, j * kTile, b);
-                tma_load_3d(sb + K0 + st * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + st], xh + 64, j * kTile, b);
-                if (j >= kStages && !(ok = mbar_wait(&bars[B_VEMPTY + st], par, abort_word, a.flags))) break;
-                mbar_expect_tx(&bars[B_VFULL + st], kTileBytes);
-                tma_load_3d(sb + V0 + st * kTileBytes, &tm_v, &bars[B_VFULL + st], xh, j * kTile, b);
-                tma_load_3d(sb + V0 + st * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + st], xh + 64, j * kTile, b);
+            for (int j = kKStages; j < n && ok; ++j) {  // Q and K_0..K_2 were issued at entry
+                const int ks = j % kKStages;
+                if (!(ok = mbar_wait(&bars[B_KEMPTY + ks], ((j / kKStages) + 1) & 1, abort_word, a.flags))) break;
+                mbar_expect_tx(&bars[B_KFULL + ks], kTileBytes);
+                tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, j * kTile, b);
+                tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64, j * kTile, b);
             }
-            // W_hi / W_lo into the K / V stages of tile n-3 once S_{n-3} / PV_{n-3}
-            // have read them (stage 2, never used, when n < 3)
+            // W_hi / W_lo (row-major, MN-major operands) into K stages freed by S_{n-3} / S_{n-2}
             const int nbh = a.B * a.H;
-            const int wst = n >= 3 ? (n - 3) % kStages : 2;
-            if (ok && n >= 3) ok = mbar_wait(&bars[B_KEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
-            if (ok && n >= 3) ok = mbar_wait(&bars[B_VEMPTY + wst], ((n - 3) / kStages) & 1, abort_word, a.flags);
+            if (ok && n >= 3) ok = mbar_wait(&bars[B_KEMPTY + wst_hi], ((n - 3) / kKStages) & 1, abort_word, a.flags);
+            if (ok && n >= 2) ok = mbar_wait(&bars[B_KEMPTY + wst_lo], ((n - 2) / kKStages) & 1, abort_word, a.flags);
             // W comes from the prep kernel, which may still be running when this
             // grid starts (programmatic dependent launch): wait for it here
             pdl_wait_primary();
             if (ok) {
                 mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
-                tma_load_3d(sb + K0 + wst * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
-                tma_load_3d(sb + K0 + wst * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
-                tma_load_3d(sb + V0 + wst * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
-                tma_load_3d(sb + V0 + wst * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
+                tma_load_3d(sb + K0 + wst_hi * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
+                tma_load_3d(sb + K0 + wst_hi * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
+                tma_load_3d(sb + K0 + wst_lo * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
+                tma_load_3d(sb + K0 + wst_lo * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
+        // S_j = Q K_j^T into S buffer j&1 (A = Q from TMEM); S_{j+2} reuses the
+        // buffer as soon as the softmax has S_j in registers, so scores run a
+        // tile ahead.  O += P_j V_j once P_j is in TMEM.
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags);
+            bool ok = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags);
             for (int j = 0; j < 2 && j < n && ok; ++j) {
-                ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags);
-                if (!ok) break;
+                if (!(ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK,
-                             kk > 0);
+                    mma_bf16_ts(tS0 + j * 128, tQ + kk * 8, kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK, kk > 0);
                 mma_commit(&bars[B_SFULL + j]);
                 mma_commit(&bars[B_KEMPTY + j]);
             }
             for (int j = 0; j < n && ok; ++j) {
-                const int sb2 = j & 1;
+                const int sbuf = j & 1;
                 if (j + 2 < n) {
-                    // S_{j+2} into S buffer j&1 once both halves have read S_j
-                    const int st2 = (j + 2) % kStages;
-                    if (!mbar_wait(&bars[B_SREAD + sb2], (j >> 1) & 1, abort_word, a.flags)) break;
-                    if (!mbar_wait(&bars[B_KFULL + st2], ((j + 2) / kStages) & 1, abort_word, a.flags)) break;
+                    const int ks = (j + 2) % kKStages;
+                    if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags))) break;
+                    if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tS0 + sb2 * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + st2 * kTileBytes, kk),
-                                 ID_KK, kk > 0);
-                    mma_commit(&bars[B_SFULL + sb2]);
-                    mma_commit(&bars[B_KEMPTY + st2]);
+                        mma_bf16_ts(tS0 + sbuf * 128, tQ + kk * 8, kmajor_desc(sb + K0 + ks * kTileBytes, kk), ID_KK,
+                                    kk > 0);
+                    mma_commit(&bars[B_SFULL + sbuf]);
+                    mma_commit(&bars[B_KEMPTY + ks]);
                 }
-                const int pb = j & 1, st = j % kStages;
-                if (!mbar_wait(&bars[B_PFULL + pb], (j >> 1) & 1, abort_word, a.flags)) break;
-                if (!mbar_wait(&bars[B_VFULL + st], (j / kStages) & 1, abort_word, a.flags)) break;
+                const int vs = j % kVStages;
+                if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags))) break;
+                if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags))) break;
                 tc_fence_after();
-                // O += P_j V_j, P_j from TMEM P buffer pb
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tO, tP0 + pb * 64 + kk * 8, mnmajor_desc(sb + V0 + st * kTileBytes, kk), ID_KMN,
-                                (j > 0 || kk > 0));
-                mma_commit(&bars[B_PVDONE + pb]);
-                mma_commit(&bars[B_VEMPTY + st]);
+                    mma_bf16_ts(tO, tP + kk * 8, mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
+                mma_commit(&bars[B_PVDONE]);
+                mma_commit(&bars[B_VEMPTY + vs]);
             }
             // O_inter = Q W_hi + Q W_lo into S buffer n&1, once S_{n-2} has been read
             if (ok && n >= 2) ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags);
             if (ok) ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags);
             if (ok) {
                 tc_fence_after();
-                const int wst = n >= 3 ? (n - 3) % kStages : 2;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), mnmajor_desc(sb + K0 + wst * kTileBytes, kk), ID_KMN,
-                             kk > 0);
+                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tOI, kmajor_desc(sb + Q, kk), mnmajor_desc(sb + V0 + wst * kTileBytes, kk), ID_KMN, 1);
+                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
                 mma_commit(&bars[B_OIDONE]);
             }
             // drain: every MMA issued so far completes before TMEM is released
@@ -231,143 +281,137 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ softmax + epilogue
-        // Warp w owns TMEM lanes (query rows) 32(w%4)..+31 and key half ch = w/4
-        // (keys 64ch..64ch+63 of each tile; output columns 64ch..64ch+63).  The
-        // two warps sharing rows exchange their half-row maxima through shared
-        // memory at a pair barrier every iteration; every wait result goes through
-        // the same exchange, so both warps always take the same path.
-        const int ch = warp >> 2;
-        const int r = (warp & 3) * 32 + lane;
-        const int pair_bar = 1 + (warp & 3);
-        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        // Thread = query row (TMEM lane); all 128 keys of a tile in registers.
+        // S_j is released (SREAD) as soon as it is in registers, so S_{j+2} is
+        // computed while this tile is exponentiated, and the registers of S_{j+1}
+        // are loaded before P_j is handed to the MMA warp.
+        //
+        // Offset: exponents are taken against a running offset m (log2 units)
+        // that is the row max of the first tile and moves only when a tile's
+        // partial sum leaves [0, 2^64): the tile is then redone against its own
+        // max, and O and l are rescaled.  Every value stays finite, P <= 2^64,
+        // and the result is the same softmax (the offset cancels in O / l).
+        const int r = warp * 32 + lane;
+        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
         const float scale = a.sm_scale_log2;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        float x[64];
-        for (int j = 0; j < n; ++j) {
-            const int s = j & 1;
-            // waits of this iteration: S_j ready; P buffer s free (PV_{j-2} done)
-            bool w_ok = ok && mbar_wait(&bars[B_SFULL + s], (j >> 1) & 1, abort_word, a.flags);
-            if (j >= 2) w_ok = w_ok && mbar_wait(&bars[B_PVDONE + s], ((j >> 1) + 1) & 1, abort_word, a.flags);
-            w_ok = __all_sync(0xffffffffu, w_ok);
-            float hm = -INFINITY;
-            if (w_ok) {
-                tc_fence_after();
-                tmem_ld32(tS0 + s * 128 + lrow + ch * 64, x);
-                tmem_ld32(tS0 + s * 128 + lrow + ch * 64 + 32, x + 32);
-                tmem_ld_wait();
-                // S_j is in registers: the MMA warp may overwrite it with S_{j+2}
-                tc_fence_before();
-                mbar_arrive(&bars[B_SREAD + s]);
-                const int valid = T - j * kTile - ch * 64;
-                if (valid < 64) {
+        float m = 0.f, l = 0.f;
+        float x[128];
+        // Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags));
+        if (!ok) {
+            // the MMA warp times out on Q as well
+        } else {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (i >= valid) x[i] = -INFINITY;
+            for (int hb = 0; hb < 2; ++hb) {
+                uint32_t qv[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hb * kHalf + sw128_offset(r, c));
+                    qv[4 * c] = v.x;
+                    qv[4 * c + 1] = v.y;
+                    qv[4 * c + 2] = v.z;
+                    qv[4 * c + 3] = v.w;
                 }
-                float m8[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) m8[k] = x[k];
-#pragma unroll
-                for (int i = 8; i < 64; i += 8)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], x[i + k]);
-                hm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                tmem_st32u(tQ + lrow + hb * 32, qv);
             }
-            xchg[(s * 2 + ch) * 128 + r] = hm;
-            xok[(s * 2 + ch) * 128 + r] = (uint8_t)w_ok;
-            named_bar_sync(pair_bar, 64);
-            ok = w_ok && xok[(s * 2 + (ch ^ 1)) * 128 + r];
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) continue;   // keep arriving at the pair barriers until the loop ends
-            const float mx = fmaxf(hm, xchg[(s * 2 + (ch ^ 1)) * 128 + r]) * scale;
-            bool rescale = false;
-            if (j == 0) {
-                m = mx;
-            } else if (mx > m + 8.0f) {
-                rescale = true;
-            }
-            if (__any_sync(0xffffffffu, rescale)) {
-                // the running max moved by more than 2^8: rescale this half of O (after PV_{j-1})
-                const bool pv_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + ((j - 1) & 1)],
-                                                                    ((j - 1) >> 1) & 1, abort_word, a.flags));
-                if (pv_ok) {
-                    tc_fence_after();
-                    const float f = rescale ? ex2(m - mx) : 1.0f;
-                    float o[32];
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        tmem_ld32(tO + lrow + ch * 64 + c * 32, o);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= f;
-                        tmem_st32(tO + lrow + ch * 64 + c * 32, o);
-                    }
-                    tmem_st_wait();
-                    if (rescale) {
-                        l *= f;
-                        m = mx;
-                    }
-                } else {
-                    ok = false;  // P_j is not written; the MMA warp times out on it
-                }
-            }
-            const float neg_m = -m;
-            // P (bf16 pairs) into this half's 32 columns of P buffer s
-            uint32_t pk[32];
-            float sum8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
-            // 1 of every 8 exponentials on the FMA pipe, the rest on MUFU; the
-            // bf16 packing on the integer pipe (MUFU is the scarce pipe here)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float e[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float arg = fmaf(x[c * 8 + k], scale, neg_m);
-                    e[k] = (k == 4) ? exp2_fma(arg) : ex2(arg);
-                    sum8[k] += e[k];
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16_rhu(e[2 * k], e[2 * k + 1]);
-            }
-            l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-            tmem_st32u(tP0 + s * 64 + lrow + ch * 32, pk);
             tmem_st_wait();
             tc_fence_before();
-            if (ok) mbar_arrive(&bars[B_PFULL + s]);
+            mbar_arrive(&bars[B_QTM]);
         }
-        // epilogue: row sum from both halves (fixed order), then this half's output columns
-        bool e_ok = ok && mbar_wait(&bars[B_PVDONE + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_word, a.flags);
-        e_ok = e_ok && mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags);
-        e_ok = __all_sync(0xffffffffu, e_ok);
-        // slot n&1 was last used in iteration n-2; the partner read it before the
-        // barrier of iteration n-1, so it is free (slot (n-1)&1 may still be read)
-        const int se = n & 1;
-        xchg[(se * 2 + ch) * 128 + r] = l;
-        xok[(se * 2 + ch) * 128 + r] = (uint8_t)e_ok;
-        named_bar_sync(pair_bar, 64);
-        e_ok = e_ok && xok[(se * 2 + (ch ^ 1)) * 128 + r];
-        e_ok = __all_sync(0xffffffffu, e_ok);
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags));
+        if (ok) {
+            tc_fence_after();
+            tmem_ld32(tS0 + lrow, x);
+            tmem_ld32(tS0 + lrow + 32, x + 32);
+            tmem_ld32(tS0 + lrow + 64, x + 64);
+            tmem_ld32(tS0 + lrow + 96, x + 96);
+        }
+        for (int j = 0; j < n && ok; ++j) {
+            const int s = j & 1;
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
+            const int valid = T - j * kTile;
+            if (valid < kTile) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= valid) x[c] = -INFINITY;
+            }
+            if (j == 0) m = row_max128(x) * scale;
+            uint32_t pk[64];
+            float lt = exp_tile(x, scale, -m, pk);
+            float f = 1.0f;
+            const bool redo = !(lt < 1.8446744e19f);  // >= 2^64, inf or NaN
+            const bool any_redo = __any_sync(0xffffffffu, redo);
+            if (any_redo) {
+                // the offset is too low for this tile (or a score is not finite):
+                // move it to the tile's max and redo P_j; O is rescaled below
+                if (redo) {
+                    const float mn = fmaxf(m, row_max128(x) * scale);
+                    f = ex2(m - mn);
+                    m = mn;
+                }
+                lt = exp_tile(x, scale, -m, pk);
+            }
+            l = fmaf(l, f, lt);
+            // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE], (j - 1) & 1, abort_word, a.flags));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            if (any_redo && j > 0) {
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 32) {
+                    float o[32];
+                    tmem_ld32(tO + lrow + c, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) o[q] *= f;
+                    tmem_st32(tO + lrow + c, o);
+                }
+            }
+            tmem_st32u(tP + lrow, pk);
+            tmem_st32u(tP + lrow + 32, pk + 32);
+            // S_{j+1} into registers while P_j is being stored
+            if (j + 1 < n) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + (s ^ 1)], ((j + 1) >> 1) & 1, abort_word,
+                                                       a.flags));
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t src = tS0 + (s ^ 1) * 128 + lrow;
+                    tmem_ld32(src, x);
+                    tmem_ld32(src + 32, x + 32);
+                    tmem_ld32(src + 64, x + 64);
+                    tmem_ld32(src + 96, x + 96);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            if (ok) mbar_arrive(&bars[B_PFULL]);
+        }
+        // epilogue: out = O / l + O_inter for this row
+        tmem_ld_wait();
+        bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags);
+        e_ok = __all_sync(0xffffffffu, e_ok && mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags));
         if (e_ok) {
             tc_fence_after();
-            const float lt = xchg[(se * 2 + 0) * 128 + r] + xchg[(se * 2 + 1) * 128 + r];
+            const float inv_l = 1.0f / l;
             const int t = q0 + r;
-            const float inv_l = 1.0f / lt;
-            const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + ch * 64;
-            float o[32], e[32];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                tmem_ld32(tO + lrow + ch * 64 + c * 32, o);
-                tmem_ld32(tOI + lrow + ch * 64 + c * 32, e);
+            const size_t row = (((size_t)b * T + t) * a.H + h) * 128;
+#pragma unroll 1
+            for (int c = 0; c < 128; c += 64) {
+                float o[64], e[64];
+                tmem_ld32(tO + lrow + c, o);
+                tmem_ld32(tO + lrow + c + 32, o + 32);
+                tmem_ld32(tOI + lrow + c, e);
+                tmem_ld32(tOI + lrow + c + 32, e + 32);
                 tmem_ld_wait();
                 if (t < T) {
                     if (a.out) {
-                        uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)a.out + row + c * 32);
+                        uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)a.out + row + c);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
+                        for (int q = 0; q < 8; ++q) {
                             uint4 w;
                             w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
                             w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
@@ -377,10 +421,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                         }
                     }
                     if (a.out_intra) {
-                        float4* di = reinterpret_cast<float4*>(a.out_intra + row + c * 32);
-                        float4* de = reinterpret_cast<float4*>(a.out_inter + row + c * 32);
+                        float4* di = reinterpret_cast<float4*>(a.out_intra + row + c);
+                        float4* de = reinterpret_cast<float4*>(a.out_inter + row + c);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
+                        for (int q = 0; q < 16; ++q) {
                             di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
                                                 o[4 * q + 3] * inv_l);
                             de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
@@ -639,8 +683,17 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
     }
     {
+        // all of a thread's gate logits are loaded before any sigmoid is taken
         float sg = 0.f;
-        for (int t = threadIdx.x; t < T; t += kThreads) sg += sigmoidf_(a.gate_logits[(size_t)bh * T + t]);
+        const float* gl = a.gate_logits + (size_t)bh * T;
+        for (int t0 = threadIdx.x; t0 < T; t0 += 8 * kThreads) {
+            float g[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) g[u] = (t0 + u * kThreads < T) ? gl[t0 + u * kThreads] : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (t0 + u * kThreads < T) sg += sigmoidf_(g[u]);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sg += __shfl_xor_sync(0xffffffffu, sg, o);
         if (lane == 0) wsum[warp] = sg;
@@ -687,20 +740,21 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         tmem_st_wait();
         // S_{N-1} row `row`, columns 64 half..+63: bf16 hi + lo into the MN-major B tiles
         park_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PARK], 0, abort_word, a.flags));
-        const float* Sp = reinterpret_cast<const float*>(smem + SPREV) + row * 128 + half * 64;
+        // float4 k of the row half is read in the order (k0 + lane) & 15, so a
+        // warp's reads (rows 512 B apart) spread over all 16-byte bank groups
+        const float4* Sp4 = reinterpret_cast<const float4*>(smem + SPREV) + row * 32 + half * 16;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float s0 = Sp[8 * c + 2 * q], s1 = Sp[8 * c + 2 * q + 1];
-                const __nv_bfloat162 hv = __floats2bfloat162_rn(s0, s1);
-                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
-                lo[q] = pack_bf16(s0 - __low2float(hv), s1 - __high2float(hv));
-            }
-            const uint32_t off = half * kHalf + sw128_offset(row, c);
-            *reinterpret_cast<uint4*>(smem + SH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(smem + SL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int k0 = 0; k0 < 16; ++k0) {
+            const int k = (k0 + lane) & 15;
+            const float4 v = Sp4[k];
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+            const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+            const uint2 hi = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+            const uint2 lo = make_uint2(pack_bf16(v.x - __low2float(h01), v.y - __high2float(h01)),
+                                        pack_bf16(v.z - __low2float(h23), v.w - __high2float(h23)));
+            const uint32_t off = half * kHalf + sw128_offset(row, k >> 1) + (k & 1) * 8;
+            *reinterpret_cast<uint2*>(smem + SH + off) = hi;
+            *reinterpret_cast<uint2*>(smem + SL + off) = lo;
         }
     } else {
         // S_{N-1} must be in shared memory before any CTA of the cluster passes the
