@@ -195,13 +195,15 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
     const uint64_t row_bytes = (uint64_t)a.H * D * 2;
     const uint64_t bh = (uint64_t)a.B * a.H;
-    CUtensorMap tq, tk, tv, tw, tphik;
+    CUtensorMap tq, tk, tv, tw, tphik, tout;
     if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+        (a.out && !map3d(&tout, a.out, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T)) ||
         !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
         !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
         !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
         !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2))
         return cudaErrorInvalidValue;
+    if (!a.out) tout = tq;  // not read: the attention kernel stores no bf16 output
     // Kernels of a pass are chained by programmatic dependent launch: prep waits
     // for the previous kernel of the stream before it reads the state, then lets
     // the attention kernel start, which reads prep's W only at its end.
@@ -226,7 +228,7 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     acfg.stream = st;
     acfg.attrs = pdl;
     acfg.numAttrs = 1;
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw, tout); });
     if (e != cudaSuccess) return e;
     if (le != cudaSuccess) return le;
     if (clean) {

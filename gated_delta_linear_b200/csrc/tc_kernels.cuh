@@ -24,10 +24,12 @@
 //   Softmax: exponents against a running offset (the first tile's row max),
 //                 moved only when a tile's partial sum leaves [0, 2^64); all
 //                 exponentials on the MUFU pipe.
-//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  At the end W_hi and
-//                 W_lo take the K stages of key tiles n-3 and n-2 (unused
+//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Near the end W_hi
+//                 and W_lo take the K stages of key tiles n-3 and n-2 (unused
 //                 stages when n < 3) and O_inter = Q W_hi + Q W_lo goes to the
-//                 S buffer the last tile does not use.
+//                 S buffer the last tile does not use while the softmax works
+//                 on the last two tiles; the bf16 output tile is assembled in
+//                 the Q buffer and written with two TMA stores.
 //   Every CTA signals at entry that the next kernel (the delta update, which
 //   reads none of this kernel's outputs) may start on idle SMs.
 //
@@ -112,7 +114,7 @@ __device__ __forceinline__ float exp_tile(const float* x, float scale, float neg
 __global__ void __launch_bounds__(attn::kThreads, 1)
     attention_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_w) {
+                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
     using namespace attn;
     extern __shared__ __align__(1024) uint8_t smem[];
     // 128B-swizzled tiles need a 1024-byte aligned base (the dynamic window starts
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
     volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+    volatile int* epi_bad = (volatile int*)(tmem_slot + 2);  // a softmax warp missed its epilogue
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -147,6 +150,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             mbar_init(&bars[i],
                       (i == B_PFULL || i == B_QTM || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads : 1);
         *abort_word = 0;
+        *epi_bad = 0;
         fence_mbar_init();
         fence_async_smem();
         tma_prefetch_desc(&tm_q);
@@ -225,13 +229,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            bool ok = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags);
+            // S_0 and S_1 take Q from shared memory (no wait for its copy into TMEM)
+            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags);
+            bool q_in_tmem = false;
             for (int j = 0; j < 2 && j < n && ok; ++j) {
                 if (!(ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tS0 + j * 128, tQ + kk * 8, kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK, kk > 0);
+                    mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK,
+                             kk > 0);
                 mma_commit(&bars[B_SFULL + j]);
                 mma_commit(&bars[B_KEMPTY + j]);
             }
@@ -239,6 +246,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 const int sbuf = j & 1;
                 if (j + 2 < n) {
                     const int ks = (j + 2) % kKStages;
+                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags))) break;
                     if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags))) break;
                     if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags))) break;
                     tc_fence_after();
@@ -249,6 +257,24 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     mma_commit(&bars[B_SFULL + sbuf]);
                     mma_commit(&bars[B_KEMPTY + ks]);
                 }
+                if (j == (n >= 2 ? n - 2 : 0)) {
+                    // O_inter = Q W_hi + Q W_lo into S buffer n&1 (free once the
+                    // softmax has S_{n-2} in registers; unused when n == 1), run
+                    // while the softmax works on the last two tiles
+                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags))) break;
+                    if (n >= 2 &&
+                        !(ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags)))
+                        break;
+                    if (!(ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
+                    mma_commit(&bars[B_OIDONE]);
+                }
                 const int vs = j % kVStages;
                 if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags))) break;
                 if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags))) break;
@@ -258,19 +284,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     mma_bf16_ts(tO, tP + kk * 8, mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
                 mma_commit(&bars[B_PVDONE]);
                 mma_commit(&bars[B_VEMPTY + vs]);
-            }
-            // O_inter = Q W_hi + Q W_lo into S buffer n&1, once S_{n-2} has been read
-            if (ok && n >= 2) ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags);
-            if (ok) ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags);
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
-                mma_commit(&bars[B_OIDONE]);
             }
             // drain: every MMA issued so far completes before TMEM is released
             mma_commit(&bars[B_Q]);
@@ -407,31 +420,41 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tmem_ld32(tOI + lrow + c, e);
                 tmem_ld32(tOI + lrow + c + 32, e + 32);
                 tmem_ld_wait();
-                if (t < T) {
-                    if (a.out) {
-                        uint4* dst = reinterpret_cast<uint4*>((__nv_bfloat16*)a.out + row + c);
+                if (a.out) {
+                    // bf16 row into the (free) Q buffer, 128B-swizzled like a TMA box
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            uint4 w;
-                            w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
-                            w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
-                            w.z = pack_bf16(o[8 * q + 4] * inv_l + e[8 * q + 4], o[8 * q + 5] * inv_l + e[8 * q + 5]);
-                            w.w = pack_bf16(o[8 * q + 6] * inv_l + e[8 * q + 6], o[8 * q + 7] * inv_l + e[8 * q + 7]);
-                            dst[q] = w;
-                        }
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
+                        w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
+                        w.z = pack_bf16(o[8 * q + 4] * inv_l + e[8 * q + 4], o[8 * q + 5] * inv_l + e[8 * q + 5]);
+                        w.w = pack_bf16(o[8 * q + 6] * inv_l + e[8 * q + 6], o[8 * q + 7] * inv_l + e[8 * q + 7]);
+                        *reinterpret_cast<uint4*>(smem + Q + (c / 64) * kHalf + sw128_offset(r, q)) = w;
                     }
-                    if (a.out_intra) {
-                        float4* di = reinterpret_cast<float4*>(a.out_intra + row + c);
-                        float4* de = reinterpret_cast<float4*>(a.out_inter + row + c);
+                }
+                if (a.out_intra && t < T) {
+                    float4* di = reinterpret_cast<float4*>(a.out_intra + row + c);
+                    float4* de = reinterpret_cast<float4*>(a.out_inter + row + c);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
-                                                o[4 * q + 3] * inv_l);
-                            de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
-                        }
+                    for (int q = 0; q < 16; ++q) {
+                        di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
+                                            o[4 * q + 3] * inv_l);
+                        de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
                     }
                 }
             }
+            if (a.out) fence_async_smem();
+        }
+        // every softmax warp reaches this barrier (no early exit); the tile is
+        // stored only if all four wrote their rows
+        if (!e_ok && lane == 0) *epi_bad = 1;
+        named_bar_sync(1, kSoftmaxThreads);
+        if (a.out && threadIdx.x == 0 && *epi_bad == 0) {
+            // rows past T are clipped by the tensor map
+            tma_store_3d(&tm_o, sb + Q, h * 128, q0, b);
+            tma_store_3d(&tm_o, sb + Q + kHalf, h * 128 + 64, q0, b);
+            bulk_commit_group();
+            bulk_wait_read_all();
         }
     }
     tc_fence_before();
@@ -616,6 +639,10 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         float x[64];
         for (int i = 0; i < nt; ++i) {
             const int s = i & 1;
+            // this row's beta logit, loaded before the wait for K~
+            const int tok = t_begin + i * kTile + r;
+            const bool valid = tok < t_end;
+            const float bl = valid ? a.beta_logits[(size_t)bh * T + tok] : 0.f;
             bool w_ok = ok && mbar_wait(&bars[B_KTFULL], i & 1, abort_word, a.flags);
             if (i > 0) w_ok = w_ok && mbar_wait(&bars[B_OPSFREE], (i - 1) & 1, abort_word, a.flags);
             w_ok = __all_sync(0xffffffffu, w_ok);
@@ -638,10 +665,8 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
             ok = __all_sync(0xffffffffu, w_ok && xok[(s * 2 + (half ^ 1)) * 128 + r]);
             if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
             const float ss = xss[(s * 2 + 0) * 128 + r] + xss[(s * 2 + 1) * 128 + r];
-            const int tok = t_begin + i * kTile + r;
-            const bool valid = tok < t_end;
             const float inv = valid ? 1.0f / sqrtf(ss + a.l2_eps) : 0.f;
-            const float beta = valid ? sigmoidf_(a.beta_logits[(size_t)bh * T + tok]) : 0.f;
+            const float beta = valid ? sigmoidf_(bl) : 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint32_t ah[4], al[4], kh[4], kl[4];
