@@ -6,11 +6,11 @@
 // inter-frame read O_inter = Q' S_{N-1}, gated delta update) and §2.2
 // (frame-level access: all tokens read the pre-update state).
 //
-// intra_frame_attention: one CTA per (128-query tile, head, batch), 7 warps.
-// Warp 4 streams Q and the K ring, warp 6 the V ring, with TMA into
-// 128B-swizzled shared memory; warp 5 issues the tcgen05 MMAs; warps 0-3 own
-// one query row per thread (a TMEM lane) and run the online softmax with all
-// 128 scores of a key tile in registers.  After the key loop the Q tile is
+// intra_frame_attention: one CTA per (128-query tile, head, batch), 11 warps.
+// Warp 8 streams Q and the K ring, warp 10 the V ring, with TMA into
+// 128B-swizzled shared memory; warp 9 issues the tcgen05 MMAs; warps 0-7 run
+// the online softmax, a query row per pair of threads (warps w and w+4, 64
+// scores each in registers).  Near the end of the key loop the Q tile is
 // multiplied by W = phi_q^T S_{N-1} (a two-term bf16 split W_hi + W_lo, row
 // major: an MN-major B operand), so the inter-frame read lands in TMEM next to
 // the softmax accumulator and the epilogue writes out = O_intra + O_inter once.
@@ -22,8 +22,8 @@
 //                 scores run a tile ahead of the softmax, and the softmax loads
 //                 S_{j+1} while it hands P_j over.
 //   Softmax: exponents against a running offset (the first tile's row max),
-//                 moved only when a tile's partial sum leaves [0, 2^64); all
-//                 exponentials on the MUFU pipe.
+//                 moved only when a tile's partial sum over a half row leaves
+//                 [0, 2^63); all exponentials on the MUFU pipe.
 //   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Near the end W_hi
 //                 and W_lo take the K stages of key tiles n-3 and n-2 (unused
 //                 stages when n < 3) and O_inter = Q W_hi + Q W_lo goes to the
@@ -63,10 +63,12 @@ constexpr uint32_t Q = 0;
 constexpr uint32_t K0 = Q + kTileBytes;
 constexpr uint32_t V0 = K0 + kKStages * kTileBytes;
 constexpr uint32_t BAR = V0 + kVStages * kTileBytes;
-constexpr uint32_t SMEM = BAR + 256;           // 229,632 B
-constexpr int kSoftmaxThreads = 128;           // warps 0-3, one query row per thread
-constexpr int kLoadWarp = 4, kMmaWarp = 5, kLoadVWarp = 6;
-constexpr int kThreads = 224;
+constexpr uint32_t XCH = BAR + 256;            // softmax pair exchange: [2 parity][2 halves][128 rows] floats
+constexpr uint32_t XFL = XCH + 2048;           // and codes [2][2][128] bytes
+constexpr uint32_t SMEM = XFL + 512;           // 232,192 B
+constexpr int kSoftmaxThreads = 256;           // warps 0-7: rows 32(w&3)..+31, column half w>>2
+constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadVWarp = 10;
+constexpr int kThreads = 352;
 enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12, B_SFULL = 15,
        B_SREAD = 17, B_QTM = 19, B_PFULL = 20, B_PVDONE = 21, B_COUNT = 22 };
 static_assert(B_COUNT * 8 + 8 <= 256, "barrier block");
@@ -82,26 +84,25 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     return sdesc_sw128(base + kk * 2048, kHalf, 1024);
 }
 
-// Row max of 128 scores (fmaxf: NaN entries are skipped).
-__device__ __forceinline__ float row_max128(const float* x) {
+// Max of N scores (fmaxf: NaN entries are skipped).
+template <int N>
+__device__ __forceinline__ float row_max(const float* x) {
     float m8[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        m8[k] = fmaxf(fmaxf(x[k], x[k + 8]), fmaxf(x[k + 16], x[k + 24]));
+    for (int k = 0; k < 8; ++k) m8[k] = x[k];
 #pragma unroll
-        for (int c = 32; c < 128; c += 32)
-            m8[k] = fmaxf(m8[k], fmaxf(fmaxf(x[c + k], x[c + k + 8]), fmaxf(x[c + k + 16], x[c + k + 24])));
-    }
+    for (int c = 8; c < N; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
     return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 
-// p = 2^(x * scale + neg_m) for one row's 128 scores, as 64 bf16 pairs (round
-// to nearest) in pk; returns the row sum of p in fp32 (the exponentials on the
-// MUFU pipe, the pair conversion one instruction per two values).
-__device__ __forceinline__ float exp_tile(const float* x, float scale, float neg_m, uint32_t* pk) {
+// p = 2^(x * scale + neg_m) for N scores, as N/2 bf16 pairs (round to
+// nearest) in pk; returns the sum of p in fp32 (the exponentials on the MUFU
+// pipe, the pair conversion one instruction per two values).
+template <int N>
+__device__ __forceinline__ float exp_scores(const float* x, float scale, float neg_m, uint32_t* pk) {
     float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < 64; ++k) {
+    for (int k = 0; k < N / 2; ++k) {
         const float e0 = ex2(fmaf(x[2 * k], scale, neg_m));
         const float e1 = ex2(fmaf(x[2 * k + 1], scale, neg_m));
         l4[(2 * k) & 3] += e0;
@@ -294,39 +295,49 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ softmax + epilogue
-        // Thread = query row (TMEM lane); all 128 keys of a tile in registers.
-        // S_j is released (SREAD) as soon as it is in registers, so S_{j+2} is
-        // computed while this tile is exponentiated, and the registers of S_{j+1}
-        // are loaded before P_j is handed to the MMA warp.
+        // Warps w and w+4 share query rows 32(w&3)..+31 (TMEM lanes); warp w>>2
+        // takes score and output columns 64(w>>2)..+63, so two softmax warps
+        // per SM sub-partition interleave their exponentials.  S_j is released
+        // (SREAD) as soon as it is in registers, so S_{j+2} is computed while
+        // this tile is exponentiated, and S_{j+1} is loaded before P_j is
+        // handed to the MMA warp.
         //
         // Offset: exponents are taken against a running offset m (log2 units)
         // that is the row max of the first tile and moves only when a tile's
-        // partial sum leaves [0, 2^64): the tile is then redone against its own
-        // max, and O and l are rescaled.  Every value stays finite, P <= 2^64,
-        // and the result is the same softmax (the offset cancels in O / l).
-        const int r = warp * 32 + lane;
-        const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+        // partial sum over a half leaves [0, 2^63): the tile is then redone
+        // against the row's max and O, l are rescaled.  Every value stays
+        // finite, P <= 2^63, and the result is the same softmax (the offset
+        // cancels in O / l).
+        //
+        // The two warps of a pair exchange a code per row and tile (0: a wait
+        // failed, 1: ok, 2: offset too low) at their pair barrier and take the
+        // same path from it; a warp whose wait failed keeps arriving at the
+        // pair barriers to the end, so neither warp ever waits for the other
+        // without a partner.
+        const int g = warp & 3, hf = warp >> 2;
+        const int r = g * 32 + lane;
+        const int pair_bar = 1 + g;
+        const uint32_t lrow = (uint32_t)(g * 32) << 16;
+        const uint32_t cs = hf * 64;
+        float* xch = (float*)(smem + XCH);
+        uint8_t* xfl = smem + XFL;
+        const int mine = hf * 128 + r, theirs = (hf ^ 1) * 128 + r;  // + parity * 256
         const float scale = a.sm_scale_log2;
         float m = 0.f, l = 0.f;
-        float x[128];
-        // Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
+        float x[64];
+        // this half of Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags));
-        if (!ok) {
-            // the MMA warp times out on Q as well
-        } else {
+        if (ok) {
+            uint32_t qv[32];
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                uint32_t qv[32];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hb * kHalf + sw128_offset(r, c));
-                    qv[4 * c] = v.x;
-                    qv[4 * c + 1] = v.y;
-                    qv[4 * c + 2] = v.z;
-                    qv[4 * c + 3] = v.w;
-                }
-                tmem_st32u(tQ + lrow + hb * 32, qv);
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hf * kHalf + sw128_offset(r, c));
+                qv[4 * c] = v.x;
+                qv[4 * c + 1] = v.y;
+                qv[4 * c + 2] = v.z;
+                qv[4 * c + 3] = v.w;
             }
+            tmem_st32u(tQ + lrow + hf * 32, qv);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[B_QTM]);
@@ -334,121 +345,141 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags));
         if (ok) {
             tc_fence_after();
-            tmem_ld32(tS0 + lrow, x);
-            tmem_ld32(tS0 + lrow + 32, x + 32);
-            tmem_ld32(tS0 + lrow + 64, x + 64);
-            tmem_ld32(tS0 + lrow + 96, x + 96);
+            tmem_ld32(tS0 + lrow + cs, x);
+            tmem_ld32(tS0 + lrow + cs + 32, x + 32);
         }
-        for (int j = 0; j < n && ok; ++j) {
+        for (int j = 0; j < n; ++j) {
             const int s = j & 1;
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
-            const int valid = T - j * kTile;
-            if (valid < kTile) {
+            const bool w_ok = ok;
+            uint32_t pk[32];
+            float lt = 0.f;
+            if (w_ok) {
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
+                const int valid = T - j * kTile - (int)cs;
+                if (valid < 64) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= valid) x[c] = -INFINITY;
+                    for (int c = 0; c < 64; ++c)
+                        if (c >= valid) x[c] = -INFINITY;
+                }
             }
-            if (j == 0) m = row_max128(x) * scale;
-            uint32_t pk[64];
-            float lt = exp_tile(x, scale, -m, pk);
-            float f = 1.0f;
-            const bool redo = !(lt < 1.8446744e19f);  // >= 2^64, inf or NaN
+            if (j == 0) {
+                // the first tile's row max over both halves sets the offset
+                const float hm = w_ok ? row_max<64>(x) : -INFINITY;
+                xch[mine] = hm;
+                named_bar_sync(pair_bar, 64);
+                m = fmaxf(hm, xch[theirs]) * scale;
+            }
+            bool redo_h = false;
+            if (w_ok) {
+                lt = exp_scores<64>(x, scale, -m, pk);
+                redo_h = !(lt < 9.2233720e18f);  // >= 2^63, inf or NaN
+            }
+            xfl[s * 256 + mine] = w_ok ? (redo_h ? 2 : 1) : 0;
+            named_bar_sync(pair_bar, 64);
+            const uint8_t pc = xfl[s * 256 + theirs];
+            ok = __all_sync(0xffffffffu, w_ok && pc != 0);  // the same in both warps of the pair
+            const bool redo = ok && (redo_h || pc == 2);
             const bool any_redo = __any_sync(0xffffffffu, redo);
+            float f = 1.0f;
             if (any_redo) {
                 // the offset is too low for this tile (or a score is not finite):
-                // move it to the tile's max and redo P_j; O is rescaled below
+                // move it to the row's max and redo P_j; O is rescaled below
+                const float hm = redo ? row_max<64>(x) * scale : -INFINITY;
+                xch[s * 256 + mine] = hm;
+                named_bar_sync(pair_bar, 64);
                 if (redo) {
-                    const float mn = fmaxf(m, row_max128(x) * scale);
+                    const float mn = fmaxf(m, fmaxf(hm, xch[s * 256 + theirs]));
                     f = ex2(m - mn);
                     m = mn;
                 }
-                lt = exp_tile(x, scale, -m, pk);
+                lt = exp_scores<64>(x, scale, -m, pk);
             }
+            if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
             l = fmaf(l, f, lt);
             // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE], (j - 1) & 1, abort_word, a.flags));
-                if (!ok) break;
+                if (!ok) continue;
                 tc_fence_after();
             }
             if (any_redo && j > 0) {
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
+                for (int c = 0; c < 64; c += 32) {
                     float o[32];
-                    tmem_ld32(tO + lrow + c, o);
+                    tmem_ld32(tO + lrow + cs + c, o);
                     tmem_ld_wait();
 #pragma unroll
                     for (int q = 0; q < 32; ++q) o[q] *= f;
-                    tmem_st32(tO + lrow + c, o);
+                    tmem_st32(tO + lrow + cs + c, o);
                 }
             }
-            tmem_st32u(tP + lrow, pk);
-            tmem_st32u(tP + lrow + 32, pk + 32);
-            // S_{j+1} into registers while P_j is being stored
+            tmem_st32u(tP + lrow + hf * 32, pk);
+            // this half of S_{j+1} into registers while P_j is being stored
             if (j + 1 < n) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + (s ^ 1)], ((j + 1) >> 1) & 1, abort_word,
                                                        a.flags));
                 if (ok) {
                     tc_fence_after();
-                    const uint32_t src = tS0 + (s ^ 1) * 128 + lrow;
+                    const uint32_t src = tS0 + (s ^ 1) * 128 + lrow + cs;
                     tmem_ld32(src, x);
                     tmem_ld32(src + 32, x + 32);
-                    tmem_ld32(src + 64, x + 64);
-                    tmem_ld32(src + 96, x + 96);
                 }
             }
             tmem_st_wait();
             tc_fence_before();
             if (ok) mbar_arrive(&bars[B_PFULL]);
         }
-        // epilogue: out = O / l + O_inter for this row
-        tmem_ld_wait();
+        // epilogue: out = O / l + O_inter for this half of the row
+        if (ok) tmem_ld_wait();
         bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags);
         e_ok = __all_sync(0xffffffffu, e_ok && mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags));
-        if (e_ok) {
+        // row sum over the two halves (slot parity n&1: its last readers passed
+        // the pair barrier of tile n-1)
+        xch[(n & 1) * 256 + mine] = l;
+        xfl[(n & 1) * 256 + mine] = e_ok ? 1 : 0;
+        named_bar_sync(pair_bar, 64);
+        const bool both = __all_sync(0xffffffffu, e_ok && xfl[(n & 1) * 256 + theirs] != 0);
+        if (both) {
             tc_fence_after();
-            const float inv_l = 1.0f / l;
+            const float inv_l = 1.0f / (l + xch[(n & 1) * 256 + theirs]);  // commutative: the same in both halves
             const int t = q0 + r;
-            const size_t row = (((size_t)b * T + t) * a.H + h) * 128;
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 64) {
-                float o[64], e[64];
-                tmem_ld32(tO + lrow + c, o);
-                tmem_ld32(tO + lrow + c + 32, o + 32);
-                tmem_ld32(tOI + lrow + c, e);
-                tmem_ld32(tOI + lrow + c + 32, e + 32);
-                tmem_ld_wait();
-                if (a.out) {
-                    // bf16 row into the (free) Q buffer, 128B-swizzled like a TMA box
+            const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + cs;
+            float o[64], e[64];
+            tmem_ld32(tO + lrow + cs, o);
+            tmem_ld32(tO + lrow + cs + 32, o + 32);
+            tmem_ld32(tOI + lrow + cs, e);
+            tmem_ld32(tOI + lrow + cs + 32, e + 32);
+            tmem_ld_wait();
+            if (a.out) {
+                // bf16 half-row into box hf of the (free) Q buffer, 128B-swizzled
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
-                        w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
-                        w.z = pack_bf16(o[8 * q + 4] * inv_l + e[8 * q + 4], o[8 * q + 5] * inv_l + e[8 * q + 5]);
-                        w.w = pack_bf16(o[8 * q + 6] * inv_l + e[8 * q + 6], o[8 * q + 7] * inv_l + e[8 * q + 7]);
-                        *reinterpret_cast<uint4*>(smem + Q + (c / 64) * kHalf + sw128_offset(r, q)) = w;
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
+                    w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
+                    w.z = pack_bf16(o[8 * q + 4] * inv_l + e[8 * q + 4], o[8 * q + 5] * inv_l + e[8 * q + 5]);
+                    w.w = pack_bf16(o[8 * q + 6] * inv_l + e[8 * q + 6], o[8 * q + 7] * inv_l + e[8 * q + 7]);
+                    *reinterpret_cast<uint4*>(smem + Q + hf * kHalf + sw128_offset(r, q)) = w;
                 }
-                if (a.out_intra && t < T) {
-                    float4* di = reinterpret_cast<float4*>(a.out_intra + row + c);
-                    float4* de = reinterpret_cast<float4*>(a.out_inter + row + c);
+                fence_async_smem();
+            }
+            if (a.out_intra && t < T) {
+                float4* di = reinterpret_cast<float4*>(a.out_intra + row);
+                float4* de = reinterpret_cast<float4*>(a.out_inter + row);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
-                                            o[4 * q + 3] * inv_l);
-                        de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
-                    }
+                for (int q = 0; q < 16; ++q) {
+                    di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
+                                        o[4 * q + 3] * inv_l);
+                    de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
                 }
             }
-            if (a.out) fence_async_smem();
         }
         // every softmax warp reaches this barrier (no early exit); the tile is
-        // stored only if all four wrote their rows
-        if (!e_ok && lane == 0) *epi_bad = 1;
-        named_bar_sync(1, kSoftmaxThreads);
+        // stored only if all eight wrote their half-rows
+        if (!both && lane == 0) *epi_bad = 1;
+        named_bar_sync(5, kSoftmaxThreads);
         if (a.out && threadIdx.x == 0 && *epi_bad == 0) {
             // rows past T are clipped by the tensor map
             tma_store_3d(&tm_o, sb + Q, h * 128, q0, b);
@@ -556,6 +587,11 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     const int t_begin = split * a.split_tokens;
     const int t_end = min(T, t_begin + a.split_tokens);
     const int nt = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+    // this thread's first gate logits (for alpha), loaded now and summed after the tile loop
+    const float* gl = a.gate_logits + (size_t)bh * T;
+    float g0[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) g0[u] = (threadIdx.x + u * kThreads < T) ? gl[threadIdx.x + u * kThreads] : 0.f;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_OPSFULL ? kNormThreads : 1);
@@ -569,6 +605,7 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tKT = tmem, tG = tmem + 128, tP = tmem + 256;
 
+    uint4 pv[8];  // phi_v staging (normalisation warps)
     // ------------------------------------------------------------ tile loop
     if (warp == kLoadWarp) {
         if (lane == 0 && nt > 0) {
@@ -692,6 +729,13 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
             tc_fence_before();
             mbar_arrive(&bars[B_OPSFULL]);
         }
+        // phi_v row r, columns 64 half..+63, loaded while the last products run
+        {
+            const uint4* src = reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.phi_v +
+                                                              (size_t)h * 128 * 128 + (size_t)r * 128 + half * 64);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) pv[c] = src[c];
+        }
         if (ok && nt > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OPSFREE], (nt - 1) & 1, abort_word, a.flags));
     }
@@ -708,10 +752,13 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
     }
     {
-        // all of a thread's gate logits are loaded before any sigmoid is taken
+        // alpha: the entry loads, then any further logits (T > 8 x 320), each
+        // batch loaded before its sigmoids are taken
         float sg = 0.f;
-        const float* gl = a.gate_logits + (size_t)bh * T;
-        for (int t0 = threadIdx.x; t0 < T; t0 += 8 * kThreads) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (threadIdx.x + u * kThreads < T) sg += sigmoidf_(g0[u]);
+        for (int t0 = threadIdx.x + 8 * kThreads; t0 < T; t0 += 8 * kThreads) {
             float g[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) g[u] = (t0 + u * kThreads < T) ? gl[t0 + u * kThreads] : 0.f;
@@ -728,17 +775,10 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         const int half = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
-        // phi_v row `row`, columns 64 half..+63, into the K-major B tile
-        {
-            const uint4* src = reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.phi_v +
-                                                              (size_t)h * 128 * 128 + (size_t)row * 128 + half * 64);
-            uint4 v[8];
+        // phi_v row `row`, columns 64 half..+63 (loaded during the tile loop), into the K-major B tile
 #pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = src[c];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(smem + PHIV + half * kHalf + sw128_offset(row, c)) = v[c];
-        }
+        for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(smem + PHIV + half * kHalf + sw128_offset(row, c)) = pv[c];
         // G and P rows `row`, columns 64 half..+63: fp32 -> bf16 hi + lo in TMEM
 #pragma unroll
         for (int gp = 0; gp < 2; ++gp) {
