@@ -123,8 +123,8 @@ cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
     static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_part[kMaxDevices],
         done_apply[kMaxDevices];
     cudaError_t e;
-    const dim3 rows(D / simt::kRows, a.H, a.B);
-    const size_t prep_smem = simt::PrepSmem<D>::bytes;
+    const dim3 rows(D / simt::prep_rows<false>(), a.H, a.B);
+    const size_t prep_smem = simt::PrepSmem<D, simt::prep_rows<false>()>::bytes;
     const size_t attn_smem = simt::AttnSmem<D>::bytes;
     const size_t ps = simt::PartialsSmem<D>::bytes;
     const size_t as = simt::ApplySmem<D, TIO>::bytes;
@@ -189,7 +189,7 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
     constexpr int D = 128;
     cudaError_t e;
-    const size_t prep_smem = simt::PrepSmem<D>::bytes;
+    const size_t prep_smem = simt::PrepSmem<D, simt::prep_rows<true>()>::bytes;
     if ((e = opt_in_smem(simt::prep_kernel<D, bf16, true>, prep_smem, done_prep)) != cudaSuccess) return e;
     if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
     if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
@@ -211,7 +211,7 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t pcfg = {};
-    pcfg.gridDim = dim3(D / simt::kRows, a.H, a.B);
+    pcfg.gridDim = dim3(D / simt::prep_rows<true>(), a.H, a.B);
     pcfg.blockDim = dim3(simt::kThreads, 1, 1);
     pcfg.dynamicSmemBytes = prep_smem;
     pcfg.stream = st;

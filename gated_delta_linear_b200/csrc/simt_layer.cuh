@@ -26,25 +26,31 @@ namespace simt {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- prep
-// grid (D/16, H, B): block x computes rows k0..k0+15 of W = phi_q^T S (row-major;
+// grid (D/R, H, B): block x computes rows k0..k0+R-1 of W = phi_q^T S (row-major;
 // fp32 for the SIMT path, a bf16 hi + lo pair for the tensor path).  S and the
-// block's 16 columns of phi_q are staged in shared memory; each warp owns two
-// rows of W and every lane D/32 consecutive columns.
+// block's R columns of phi_q are staged in shared memory; each warp owns R/8
+// rows of W and every lane D/32 consecutive columns.  The tensor path takes
+// R = 64 (two blocks per head), so that the attention kernel launched behind it
+// finds most SMs free; the SIMT path takes R = 16.
 constexpr int kRows = 16;
+template <bool kSplitOut>
+__host__ __device__ constexpr int prep_rows() { return kSplitOut ? 64 : 16; }
 
-template <int D>
+template <int D, int R>
 struct PrepSmem {
-    static constexpr size_t bytes = sizeof(float) * (D * D + D * kRows + kRows * (D + 1));
+    static constexpr size_t bytes = sizeof(float) * (D * D + D * R);
 };
 
 template <int D, typename TIO, bool kSplitOut>
 __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) {
     constexpr int NC = D / 32;
+    constexpr int R = prep_rows<kSplitOut>();
+    constexpr int RW = R / (kThreads / 32);  // rows of W per warp
+    static_assert(RW == 2 || RW % 4 == 0, "rows per warp");
     extern __shared__ float smem[];
-    float* Ss = smem;                  // [D][D]     S_{N-1}
-    float* Ph = Ss + D * D;            // [D][16]    phi_q[o][k0 + kr]
-    float* Wst = Ph + D * kRows;       // [16][D+1]  W rows (for the transposed split store)
-    const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * kRows;
+    float* Ss = smem;                  // [D][D]  S_{N-1}
+    float* Ph = Ss + D * D;            // [D][R]  phi_q[o][k0 + kr]
+    const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * R;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
     if constexpr (kSplitOut) {
@@ -63,12 +69,12 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
 #pragma unroll
         for (int u = 0; u < NS; ++u) sv[u] = S4[tid + u * kThreads];
         const TIO* phiq = (const TIO*)a.phi_q + (size_t)h * D * D;
-        constexpr int NP = D * kRows / kThreads;
+        constexpr int NP = D * R / kThreads;
         float pv[NP];
 #pragma unroll
         for (int u = 0; u < NP; ++u) {
             const int i = tid + u * kThreads;
-            pv[u] = to_f32(phiq[(i / kRows) * D + k0 + i % kRows]);
+            pv[u] = to_f32(phiq[(i / R) * D + k0 + i % R]);
         }
 #pragma unroll
         for (int u = 0; u < NS; ++u) reinterpret_cast<float4*>(Ss)[tid + u * kThreads] = sv[u];
@@ -76,25 +82,40 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
         for (int u = 0; u < NP; ++u) Ph[tid + u * kThreads] = pv[u];
     }
     __syncthreads();
-    // each warp owns rows r0, r0+1 of W; each lane NC consecutive columns
-    const int r0 = 2 * warp;
-    float acc[2][NC];
+    // each warp owns rows r0..r0+RW-1 of W; each lane NC consecutive columns
+    const int r0 = RW * warp;
+    float acc[RW][NC];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) acc[0][c] = acc[1][c] = 0.f;
+    for (int q = 0; q < RW; ++q)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) acc[q][c] = 0.f;
 #pragma unroll 4
     for (int o = 0; o < D; ++o) {
-        const float2 p = *reinterpret_cast<const float2*>(Ph + o * kRows + r0);
+        float p[RW];
+        if constexpr (RW == 2) {
+            const float2 p2 = *reinterpret_cast<const float2*>(Ph + o * R + r0);
+            p[0] = p2.x;
+            p[1] = p2.y;
+        } else {
+#pragma unroll
+            for (int q = 0; q < RW; q += 4) {
+                const float4 p4 = *reinterpret_cast<const float4*>(Ph + o * R + r0 + q);
+                p[q] = p4.x;
+                p[q + 1] = p4.y;
+                p[q + 2] = p4.z;
+                p[q + 3] = p4.w;
+            }
+        }
         float sv[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) sv[c] = Ss[o * D + NC * lane + c];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            acc[0][c] = fmaf(p.x, sv[c], acc[0][c]);
-            acc[1][c] = fmaf(p.y, sv[c], acc[1][c]);
-        }
+        for (int q = 0; q < RW; ++q)
+#pragma unroll
+            for (int c = 0; c < NC; ++c) acc[q][c] = fmaf(p[q], sv[c], acc[q][c]);
     }
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
+    for (int rr = 0; rr < RW; ++rr) {
         const size_t row = bh * D * D + (size_t)(k0 + r0 + rr) * D + NC * lane;
         if constexpr (kSplitOut) {
             // row-major W as a bf16 hi + lo pair
@@ -117,7 +138,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
     if (clean && !kSplitOut) {
         // the fp32 update reads S_{N-1} from this copy (it writes the state in place)
         float4* dst = reinterpret_cast<float4*>(a.S_prev + bh * D * D + (size_t)k0 * D);
-        for (int i = tid; i < kRows * D / 4; i += kThreads)
+        for (int i = tid; i < R * D / 4; i += kThreads)
             dst[i] = reinterpret_cast<const float4*>(Ss + k0 * D)[i];
     }
 }
