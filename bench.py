@@ -47,6 +47,9 @@ def _args():
     p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     p.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layer", choices=["hybrid", "kvcache"], default="hybrid",
+                   help="hybrid: the ARL2 layer (the reported benchmark); kvcache: the softmax "
+                        "baseline with a growing key/value cache on the same stream, for comparison")
     p.add_argument("--profile-run", action="store_true",
                    help="3 warm-up frames then one frame of the 480p workload; no JSON line "
                         "(a small, fixed launch sequence for ncu captures)")
@@ -396,10 +399,77 @@ def _src_hash():
     return h.hexdigest()[:16]
 
 
+def run_kvcache(args):
+    """The softmax baseline with a key/value cache on the 480p stream: frame N
+    attends over frames 0..N (ARL2 summary §1; §4 compares against it).  Times
+    the 21-frame stream with CUDA events on one GPU (inputs resident), reports
+    the first and last frames' times and the cache's size next to the hybrid
+    layer's constant state."""
+    import torch
+    import gated_delta_linear_b200 as G
+    import workloads as W
+
+    w = W.WORKLOADS[1]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    frames = []
+    for n in range(w.frames):
+        x = W.pass_inputs(w, n, 0)
+        frames.append([t.to(dev) for t in (x.q, x.k, x.v)])
+    layer = G.KVCacheAttention(w.B, w.H, w.T, w.d, w.frames, device=dev)
+    outs = [torch.empty_like(f[0]) for f in frames]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.reset()
+        for f, o in zip(frames, outs):
+            layer.forward(*f, out=o)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    steps = max(1, args.steps // 10)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        start.record(stream)
+        for _ in range(steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(stop)
+    # per-frame times of one more step, frame by frame
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.frames + 1)]
+    layer.reset()
+    ev[0].record(stream)
+    for i, (f, o) in enumerate(zip(frames, outs)):
+        layer.forward(*f, out=o)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    per_frame = [ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(w.frames)]
+    assert layer.device_status() == G.HYB_OK
+    tokens = w.B * w.T * w.frames
+    line = {
+        "layer": "kvcache_softmax_baseline",
+        "metric": "softmax + KV-cache layer tokens/s (21-frame 480p forward, 1 B200)",
+        "value": tokens * steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms / steps, "us_per_frame": ms / steps / w.frames * 1e3,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded normals, video-DiT shapes)",
+        "config": _config(w, {"layer": "softmax attention over all cached frames (no state)"}),
+        "us_first_frame": per_frame[0], "us_last_frame": per_frame[-1],
+        "kv_cache_bytes_after_last_frame": layer.cache_bytes(),
+        "hybrid_state_bytes": w.B * w.H * w.d * w.d * 4,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.layer == "kvcache":
+        return run_kvcache(args)
     return run_cuda(args)
 
 

@@ -30,7 +30,9 @@ from ._binding import (  # noqa: F401
     HYB_NOALLOC_SCRATCH_BYTES,
     hyb_attn_get_device_status,
     hyb_attn_status_string,
+    hyb_kvcache_attn_forward,
     HybridAttention,
+    KVCacheAttention,
     HybAttnTiming,
     HYB_NUM_KERNELS,
     hyb_attn_timing_begin,

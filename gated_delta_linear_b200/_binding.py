@@ -60,6 +60,8 @@ def _load():
     L.hyb_attn_forward_branches.restype = i
     L.hyb_attn_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
     L.hyb_attn_forward_noalloc.restype = i
+    L.hyb_kvcache_attn_forward.argtypes = [dp, vp, vp, vp, vp, vp, i, i, vp, vp, sz, vp]
+    L.hyb_kvcache_attn_forward.restype = i
     L.hyb_attn_get_device_status.argtypes = [vp, vp]
     L.hyb_attn_get_device_status.restype = i
     L.hyb_attn_timing_begin.argtypes = [i]
@@ -136,6 +138,15 @@ def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, be
                                         _stream(stream))
 
 
+def hyb_kvcache_attn_forward(desc, q, k, v, k_cache, v_cache, cache_tokens, cached_tokens, out,
+                             workspace, workspace_bytes=None, stream=None) -> int:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_kvcache_attn_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache),
+                                        _ptr(v_cache), int(cache_tokens), int(cached_tokens), _ptr(out),
+                                        _ptr(workspace), workspace_bytes, _stream(stream))
+
+
 def hyb_attn_get_device_status(workspace, stream=None) -> int:
     return lib.hyb_attn_get_device_status(_ptr(workspace), _stream(stream))
 
@@ -204,6 +215,44 @@ class HybridAttention:
         if st != HYB_OK:
             raise HybAttnError(st, "hyb_attn_forward_branches")
         return out, oi, oe
+
+    def device_status(self, stream=None) -> int:
+        return hyb_attn_get_device_status(self.workspace, stream)
+
+
+class KVCacheAttention:
+    """The softmax baseline with a growing key/value cache: owns the bf16 caches
+    [B, max_frames * T, H, d] and a status workspace; ``forward`` marshals one
+    frame into ``hyb_kvcache_attn_forward`` (which appends the frame's k, v and
+    attends over every cached token) and advances the cached-token count."""
+
+    def __init__(self, B, H, T, d, max_frames, device="cuda", sm_scale=0.0):
+        import torch
+        self.desc = make_desc(B, H, T, d, HYB_BF16, sm_scale)
+        self.device = torch.device(device)
+        self.capacity = max_frames * T
+        self.k_cache = torch.zeros(B, self.capacity, H, d, dtype=torch.bfloat16, device=self.device)
+        self.v_cache = torch.zeros_like(self.k_cache)
+        self.workspace = torch.zeros(256, dtype=torch.uint8, device=self.device)
+        self.cached = 0
+
+    def reset(self):
+        self.cached = 0
+
+    def cache_bytes(self) -> int:
+        """Bytes of key/value cache in use."""
+        return 2 * self.k_cache.shape[0] * self.cached * self.k_cache.shape[2] * self.k_cache.shape[3] * 2
+
+    def forward(self, q, k, v, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        st = hyb_kvcache_attn_forward(self.desc, q, k, v, self.k_cache, self.v_cache, self.capacity,
+                                      self.cached, out, self.workspace, stream=stream)
+        if st != HYB_OK:
+            raise HybAttnError(st, "hyb_kvcache_attn_forward")
+        self.cached += q.shape[1]
+        return out
 
     def device_status(self, stream=None) -> int:
         return hyb_attn_get_device_status(self.workspace, stream)

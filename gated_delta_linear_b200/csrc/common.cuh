@@ -17,6 +17,8 @@ constexpr size_t kStatusBytes = 256;  // status block at the start of the worksp
 // Everything one pass needs; built on the host from the C-ABI arguments.
 struct LayerArgs {
     int B, H, T, D;
+    int T_kv;              // keys the attention kernel reads (T, or the cached tokens of a KV cache)
+    int inter;             // 1: the attention kernel adds O_inter = Q W (hybrid layer); 0: softmax only
     float sm_scale_log2;   // softmax scale * log2(e)
     float l2_eps;
     const void* q;

@@ -280,6 +280,8 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.B = desc->B;
     a.H = desc->H;
     a.T = desc->T;
+    a.T_kv = desc->T;
+    a.inter = 1;
     a.D = p.D;
     const float scale = desc->sm_scale > 0.f ? desc->sm_scale : 1.0f / sqrtf((float)desc->d_k);
     a.sm_scale_log2 = scale * 1.4426950408889634f;
@@ -315,9 +317,89 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
+// Softmax attention of one frame's queries over a KV cache (the baseline the
+// hybrid layer replaces): append the frame's k, v at row `cached` of each
+// batch's cache, then run the attention kernel over cached + T keys with no
+// inter-frame read.
+hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v, void* k_cache,
+                        void* v_cache, int cache_tokens, int cached_tokens, void* out, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+    if (!desc) return HYB_ERR_INVALID;
+    if (desc->B <= 0 || desc->H <= 0 || desc->T <= 0 || desc->d_k <= 0 || desc->d_v <= 0) return HYB_ERR_INVALID;
+    if (desc->dtype != HYB_BF16 && desc->dtype != HYB_FP32) return HYB_ERR_INVALID;
+    if (!isfinite(desc->sm_scale)) return HYB_ERR_INVALID;
+    if (desc->dtype != HYB_BF16 || desc->d_k != 128 || desc->d_v != 128) return HYB_ERR_UNSUPPORTED;
+    if (desc->H > 65535 || desc->B > 65535) return HYB_ERR_UNSUPPORTED;
+    if (cached_tokens < 0 || cache_tokens <= 0 || (long long)cached_tokens + desc->T > cache_tokens)
+        return HYB_ERR_INVALID;
+    if ((double)desc->B * cache_tokens * desc->H * 128 >= 2147483647.0) return HYB_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !k_cache || !v_cache || !out) return HYB_ERR_INVALID;
+    const void* ptrs[] = {q, k, v, k_cache, v_cache, out, workspace};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return HYB_ERR_ALIGN;
+    if (!workspace || workspace_bytes < kStatusBytes) return HYB_ERR_WORKSPACE;
+
+    constexpr int D = 128;
+    const int B = desc->B, H = desc->H, T = desc->T;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t row = (size_t)H * D;  // elements per token row
+    for (int b = 0; b < B; ++b) {
+        const size_t dst = ((size_t)b * cache_tokens + cached_tokens) * row * 2;
+        const size_t src = (size_t)b * T * row * 2;
+        if (cudaMemcpyAsync((char*)k_cache + dst, (const char*)k + src, (size_t)T * row * 2,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync((char*)v_cache + dst, (const char*)v + src, (size_t)T * row * 2,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return HYB_ERR_CUDA;
+    }
+    LayerArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.H = H;
+    a.T = T;
+    a.T_kv = cached_tokens + T;
+    a.inter = 0;
+    a.D = D;
+    const float scale = desc->sm_scale > 0.f ? desc->sm_scale : 1.0f / sqrtf((float)desc->d_k);
+    a.sm_scale_log2 = scale * 1.4426950408889634f;
+    a.q = q;
+    a.k = k_cache;
+    a.v = v_cache;
+    a.out = out;
+    a.flags = (unsigned*)workspace;
+
+    static unsigned char done_attn[kMaxDevices];
+    cudaError_t e;
+    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
+    const uint64_t row_bytes = (uint64_t)H * D * 2;
+    CUtensorMap tq, tk, tv, tout;
+    if (!map3d(&tq, q, (uint64_t)H * D, T, B, row_bytes, row_bytes * T) ||
+        !map3d(&tk, k_cache, (uint64_t)H * D, a.T_kv, B, row_bytes, row_bytes * cache_tokens) ||
+        !map3d(&tv, v_cache, (uint64_t)H * D, a.T_kv, B, row_bytes, row_bytes * cache_tokens) ||
+        !map3d(&tout, out, (uint64_t)H * D, T, B, row_bytes, row_bytes * T))
+        return HYB_ERR_CUDA;
+    cudaLaunchConfig_t acfg = {};
+    acfg.gridDim = dim3((T + tc::kTile - 1) / tc::kTile, H, B);
+    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::attn::SMEM;
+    acfg.stream = st;
+    cudaError_t le = cudaSuccess;
+    // tq stands in for the unused W map
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
+    if (e != cudaSuccess || le != cudaSuccess) return HYB_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+hyb_status hyb_kvcache_attn_forward(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                                    void* k_cache, void* v_cache, int cache_tokens, int cached_tokens, void* out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return kvcache_impl(desc, q, k, v, k_cache, v_cache, cache_tokens, cached_tokens, out, workspace,
+                        workspace_bytes, stream);
+}
 
 size_t hyb_attn_workspace_bytes(const hyb_attn_desc* desc) {
     Plan p;

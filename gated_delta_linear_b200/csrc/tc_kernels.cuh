@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T;
     const int q0 = qt_ * kTile;
-    const int n = (T + kTile - 1) / kTile;
+    const int n = (a.T_kv + kTile - 1) / kTile;  // key tiles
+    const bool inter = a.inter != 0;             // add O_inter = Q W (hybrid layer)
     const int bh = b * a.H + h;
     // K stages that receive W_hi / W_lo at the end (free once the scores of key
     // tiles n-3 / n-2 are computed; stages no tile uses when n is small)
@@ -208,12 +209,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             }
             // W_hi / W_lo (row-major, MN-major operands) into K stages freed by S_{n-3} / S_{n-2}
             const int nbh = a.B * a.H;
-            if (ok && n >= 3) ok = mbar_wait(&bars[B_KEMPTY + wst_hi], ((n - 3) / kKStages) & 1, abort_word, a.flags);
-            if (ok && n >= 2) ok = mbar_wait(&bars[B_KEMPTY + wst_lo], ((n - 2) / kKStages) & 1, abort_word, a.flags);
+            if (inter && ok && n >= 3)
+                ok = mbar_wait(&bars[B_KEMPTY + wst_hi], ((n - 3) / kKStages) & 1, abort_word, a.flags);
+            if (inter && ok && n >= 2)
+                ok = mbar_wait(&bars[B_KEMPTY + wst_lo], ((n - 2) / kKStages) & 1, abort_word, a.flags);
             // W comes from the prep kernel, which may still be running when this
             // grid starts (programmatic dependent launch): wait for it here
-            pdl_wait_primary();
-            if (ok) {
+            if (inter) pdl_wait_primary();
+            if (inter && ok) {
                 mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
                 tma_load_3d(sb + K0 + wst_hi * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
                 tma_load_3d(sb + K0 + wst_hi * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     mma_commit(&bars[B_SFULL + sbuf]);
                     mma_commit(&bars[B_KEMPTY + ks]);
                 }
-                if (j == (n >= 2 ? n - 2 : 0)) {
+                if (inter && j == (n >= 2 ? n - 2 : 0)) {
                     // O_inter = Q W_hi + Q W_lo into S buffer n&1 (free once the
                     // softmax has S_{n-2} in registers; unused when n == 1), run
                     // while the softmax works on the last two tiles
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
-                const int valid = T - j * kTile - (int)cs;
+                const int valid = a.T_kv - j * kTile - (int)cs;
                 if (valid < 64) {
 #pragma unroll
                     for (int c = 0; c < 64; ++c)
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // epilogue: out = O / l + O_inter for this half of the row
         if (ok) tmem_ld_wait();
         bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags);
-        e_ok = __all_sync(0xffffffffu, e_ok && mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags));
+        e_ok = __all_sync(0xffffffffu, e_ok && (!inter || mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags)));
         // row sum over the two halves (slot parity n&1: its last readers passed
         // the pair barrier of tile n-1)
         xch[(n & 1) * 256 + mine] = l;
@@ -449,8 +452,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             float o[64], e[64];
             tmem_ld32(tO + lrow + cs, o);
             tmem_ld32(tO + lrow + cs + 32, o + 32);
-            tmem_ld32(tOI + lrow + cs, e);
-            tmem_ld32(tOI + lrow + cs + 32, e + 32);
+            if (inter) {
+                tmem_ld32(tOI + lrow + cs, e);
+                tmem_ld32(tOI + lrow + cs + 32, e + 32);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 64; ++q) e[q] = 0.f;
+            }
             tmem_ld_wait();
             if (a.out) {
                 // bf16 half-row into box hf of the (free) Q buffer, 128B-swizzled

@@ -139,6 +139,30 @@ hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc,
                                     const float* gate_logits, const float* beta_logits,
                                     float* state, int clean_pass, void* out, void* stream);
 
+/* hyb_kvcache_attn_forward -- the softmax baseline the hybrid layer replaces
+ * (ARL2 summary §1, problem statement: softmax self-attention whose key/value
+ * cache grows with every generated chunk; §4, the memory and wall-clock
+ * comparison against it).  One call per frame: the frame's k and v
+ * ([B][T][H][128] bf16) are copied into rows [cached_tokens, cached_tokens+T)
+ * of each batch's cache, then every query of the frame attends, with softmax
+ * scale desc->sm_scale (<= 0: 1/sqrt(128)), over all cached_tokens + T keys:
+ *     out = softmax(q k_cache^T * scale) v_cache,
+ * bidirectional within the frame and over every earlier frame, no inter-frame
+ * read and no state.  The caller tracks cached_tokens (0 for the first frame;
+ * add T after each call).
+ *   k_cache, v_cache: [B][cache_tokens][H][128] bf16, caller-owned; rows
+ *       >= cached_tokens + T are never read.
+ *   out: [B][T][H][128] bf16.  workspace: at least 256 bytes, zero-filled once
+ *       (device status flags, read by hyb_attn_get_device_status).
+ * desc: B, H, T, d_k = d_v = 128, dtype HYB_BF16 (else HYB_ERR_UNSUPPORTED);
+ * l2_eps is ignored.  HYB_ERR_INVALID if cached_tokens < 0 or
+ * cached_tokens + T > cache_tokens; HYB_ERR_ALIGN if a pointer is not 16-byte
+ * aligned; HYB_ERR_WORKSPACE if the workspace is missing or too small.
+ * Asynchronous on `stream`, like hyb_attn_forward. */
+hyb_status hyb_kvcache_attn_forward(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                                    void* k_cache, void* v_cache, int cache_tokens, int cached_tokens,
+                                    void* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status flags kept
  * in `workspace`: HYB_ERR_CUDA if a kernel found its launch environment
  * unusable (e.g. a misaligned shared-memory window) and did nothing,

@@ -8,7 +8,8 @@ or helpers with ``gated_delta_linear_b200``, and neither side imports the other.
 
 Source: "Technical summary: Attend Locally, Remember Linearly (ARL2)"
 (gist.science/ar/paper/2605.16579), §2.1 "hybrid attention decomposition"
-and §2.2 "memory-state management".
+and §2.2 "memory-state management"; §1 for the key/value-cache softmax
+baseline (``kvcache_attention``).
 """
 
 from .hybrid_layer import (  # noqa: F401
@@ -22,4 +23,5 @@ from .hybrid_layer import (  # noqa: F401
     head_pass,
     layer_pass,
     run_frames,
+    kvcache_attention,
 )

@@ -216,3 +216,25 @@ def run_frames(frame_source, phi_q, phi_k, phi_v, state0, n_frames, passes,
                 on_pass(n, p, out, oi, oe, state, new_state)
             state = new_state
     return state
+
+
+def kvcache_attention(q, k_frames, v_frames, sm_scale):
+    """The softmax baseline with a key/value cache, for one frame of one head.
+
+    ARL2 summary §1 (problem statement): the softmax attention of an
+    autoregressive video DiT keeps the keys and values of every generated chunk
+    in a cache that grows linearly with the video; §4 compares the hybrid layer's
+    memory and wall-clock time against it.  The queries of frame N attend,
+    with one softmax, over the keys of frames 0..N (bidirectional within frame
+    N, no mask): the cache is the frames' keys and values stacked in order.
+    q: [T, d] of frame N; k_frames, v_frames: sequences of [T_f, d] for frames
+    0..N.  Returns [T, d].
+    """
+    k = np.concatenate([np.asarray(x, dtype=np.float64) for x in k_frames], axis=0)
+    v = np.concatenate([np.asarray(x, dtype=np.float64) for x in v_frames], axis=0)
+    q = np.asarray(q, dtype=np.float64)
+    scores = (q @ k.T) * sm_scale
+    scores = scores - scores.max(axis=1, keepdims=True)
+    weights = np.exp(scores)
+    weights = weights / weights.sum(axis=1, keepdims=True)
+    return weights @ v

@@ -100,3 +100,26 @@ def test_desc_layout_matches_header():
     assert ctypes.sizeof(G.HybAttnDesc) == 32
     names = [f[0] for f in G.HybAttnDesc._fields_]
     assert names == ["B", "H", "T", "d_k", "d_v", "dtype", "sm_scale", "l2_eps"]
+
+
+def test_kvcache_host_validation_rejects_before_launch():
+    d = G.make_desc(1, 12, 1560, 128)
+    ws = FAKE
+
+    def call(desc=d, cache=4 * 1560, cached=0, **over):
+        args = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, out=FAKE, ws=ws, nbytes=256)
+        args.update(over)
+        return G.lib.hyb_kvcache_attn_forward(ctypes.byref(desc), args["q"], args["k"], args["v"], args["kc"],
+                                              args["vc"], cache, cached, args["out"], args["ws"],
+                                              args["nbytes"], None)
+
+    assert G.lib.hyb_kvcache_attn_forward(None, *([None] * 5), 1, 0, None, None, 0, None) == G.HYB_ERR_INVALID
+    assert call(cached=3 * 1560 + 1) == G.HYB_ERR_INVALID      # the frame would overflow the cache
+    assert call(cached=-1) == G.HYB_ERR_INVALID
+    assert call(q=None) == G.HYB_ERR_INVALID
+    assert call(vc=None) == G.HYB_ERR_INVALID
+    assert call(desc=G.make_desc(1, 12, 1560, 64)) == G.HYB_ERR_UNSUPPORTED
+    assert call(desc=G.make_desc(1, 2, 64, 32, G.HYB_FP32)) == G.HYB_ERR_UNSUPPORTED
+    assert call(kc=FAKE + 8) == G.HYB_ERR_ALIGN
+    assert call(ws=None) == G.HYB_ERR_WORKSPACE
+    assert call(nbytes=255) == G.HYB_ERR_WORKSPACE
