@@ -31,6 +31,7 @@ from ._binding import (  # noqa: F401
     hyb_attn_get_device_status,
     hyb_attn_status_string,
     hyb_kvcache_attn_forward,
+    hyb_attn_forward_mixed,
     HybridAttention,
     KVCacheAttention,
     HybAttnTiming,

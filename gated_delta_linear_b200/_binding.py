@@ -60,6 +60,8 @@ def _load():
     L.hyb_attn_forward_branches.restype = i
     L.hyb_attn_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
     L.hyb_attn_forward_noalloc.restype = i
+    L.hyb_attn_forward_mixed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
+    L.hyb_attn_forward_mixed.restype = i
     L.hyb_kvcache_attn_forward.argtypes = [dp, vp, vp, vp, vp, vp, i, i, vp, vp, sz, vp]
     L.hyb_kvcache_attn_forward.restype = i
     L.hyb_attn_get_device_status.argtypes = [vp, vp]
@@ -136,6 +138,16 @@ def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, be
                                         _ptr(phi_q), _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits),
                                         _ptr(beta_logits), _ptr(state), int(clean_pass), _ptr(out),
                                         _stream(stream))
+
+
+def hyb_attn_forward_mixed(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                           clean_pass, mix, out, workspace, workspace_bytes=None, stream=None) -> int:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_attn_forward_mixed(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(phi_q),
+                                      _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits), _ptr(beta_logits),
+                                      _ptr(state), int(clean_pass), _ptr(mix), _ptr(out), _ptr(workspace),
+                                      workspace_bytes, _stream(stream))
 
 
 def hyb_kvcache_attn_forward(desc, q, k, v, k_cache, v_cache, cache_tokens, cached_tokens, out,
@@ -215,6 +227,17 @@ class HybridAttention:
         if st != HYB_OK:
             raise HybAttnError(st, "hyb_attn_forward_branches")
         return out, oi, oe
+
+    def forward_mixed(self, q, k, v, gate_logits, beta_logits, clean_pass, mix, out=None, stream=None):
+        """out = a O_intra + c O_inter with (a, c) = mix[b, h] ([B, H, 2] fp32 on the device)."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        st = hyb_attn_forward_mixed(self.desc, q, k, v, *self.phi, gate_logits, beta_logits, self.state,
+                                    clean_pass, mix, out, self.workspace, stream=stream)
+        if st != HYB_OK:
+            raise HybAttnError(st, "hyb_attn_forward_mixed")
+        return out
 
     def device_status(self, stream=None) -> int:
         return hyb_attn_get_device_status(self.workspace, stream)

@@ -19,6 +19,7 @@ struct LayerArgs {
     int B, H, T, D;
     int T_kv;              // keys the attention kernel reads (T, or the cached tokens of a KV cache)
     int inter;             // 1: the attention kernel adds O_inter = Q W (hybrid layer); 0: softmax only
+    const float* mix;      // [B][H][2] (a, c): out = a O_intra + c O_inter; NULL: a = c = 1
     float sm_scale_log2;   // softmax scale * log2(e)
     float l2_eps;
     const void* q;

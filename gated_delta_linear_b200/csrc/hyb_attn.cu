@@ -260,7 +260,7 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
                         const void* phi_q, const void* phi_k, const void* phi_v,
                         const float* gate_logits, const float* beta_logits, float* state,
                         int clean_pass, void* out, float* out_intra, float* out_inter,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+                        void* workspace, size_t workspace_bytes, void* stream, const float* mix = nullptr) {
     Plan p;
     hyb_status s = make_plan(desc, &p);
     if (s != HYB_OK) return s;
@@ -270,7 +270,7 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     if ((out_intra == nullptr) != (out_inter == nullptr)) return HYB_ERR_INVALID;
     if (clean_pass && (!gate_logits || !beta_logits)) return HYB_ERR_INVALID;
     const void* ptrs[] = {q, k, v, phi_q, phi_k, phi_v, state, out, out_intra, out_inter,
-                          gate_logits, beta_logits, workspace};
+                          gate_logits, beta_logits, workspace, mix};
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return HYB_ERR_ALIGN;
     if (!workspace || workspace_bytes < p.total) return HYB_ERR_WORKSPACE;
@@ -282,6 +282,7 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.T = desc->T;
     a.T_kv = desc->T;
     a.inter = 1;
+    a.mix = mix;
     a.D = p.D;
     const float scale = desc->sm_scale > 0.f ? desc->sm_scale : 1.0f / sqrtf((float)desc->d_k);
     a.sm_scale_log2 = scale * 1.4426950408889634f;
@@ -425,6 +426,16 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc, const void* q, c
     if (!out_intra || !out_inter) return HYB_ERR_INVALID;
     return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
                         clean_pass, out, out_intra, out_inter, workspace, workspace_bytes, stream);
+}
+
+hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                                  const void* phi_q, const void* phi_k, const void* phi_v,
+                                  const float* gate_logits, const float* beta_logits, float* state,
+                                  int clean_pass, const float* mix, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    if (!mix || !out) return HYB_ERR_INVALID;
+    return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out,
+                        nullptr, nullptr, workspace, workspace_bytes, stream, mix);
 }
 
 hyb_status hyb_attn_get_device_status(const void* workspace, void* stream) {

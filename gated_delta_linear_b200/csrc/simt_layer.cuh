@@ -114,6 +114,14 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
 #pragma unroll
             for (int c = 0; c < NC; ++c) acc[q][c] = fmaf(p[q], sv[c], acc[q][c]);
     }
+    // branch combination: the inter-frame gain c folds into W (Q (c W) = c O_inter)
+    if (a.mix) {
+        const float cg = a.mix[bh * 2 + 1];
+#pragma unroll
+        for (int q = 0; q < RW; ++q)
+#pragma unroll
+            for (int c = 0; c < NC; ++c) acc[q][c] *= cg;
+    }
 #pragma unroll
     for (int rr = 0; rr < RW; ++rr) {
         const size_t row = bh * D * D + (size_t)(k0 + r0 + rr) * D + NC * lane;
@@ -224,6 +232,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(LayerArgs a) {
     }
     // inter-frame read: O_inter = Q (phi_q^T S)
     const float* W = a.W + ((size_t)b * a.H + h) * D * D;
+    const float ag = a.mix ? a.mix[((size_t)b * a.H + h) * 2] : 1.0f;  // weight of O_intra in out
     float oe[8][NC];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
@@ -251,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(LayerArgs a) {
             const int col = lane + 32 * c;
             const float intra = o[r][c] * inv_l;
             const float inter = oe[r][c];
-            if (a.out) ((TIO*)a.out)[row + col] = from_f32<TIO>(intra + inter);
+            if (a.out) ((TIO*)a.out)[row + col] = from_f32<TIO>(fmaf(ag, intra, inter));
             if (a.out_intra) a.out_intra[row + col] = intra;
             if (a.out_inter) a.out_inter[row + col] = inter;
         }

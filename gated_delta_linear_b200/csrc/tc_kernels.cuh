@@ -447,6 +447,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (both) {
             tc_fence_after();
             const float inv_l = 1.0f / (l + xch[(n & 1) * 256 + theirs]);  // commutative: the same in both halves
+            // out = a O_intra + O_inter (the inter gain c is folded into W); a = 1 without a mix
+            const float inv_out = a.mix ? inv_l * a.mix[bh * 2] : inv_l;
             const int t = q0 + r;
             const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + cs;
             float o[64], e[64];
@@ -465,10 +467,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint4 w;
-                    w.x = pack_bf16(o[8 * q + 0] * inv_l + e[8 * q + 0], o[8 * q + 1] * inv_l + e[8 * q + 1]);
-                    w.y = pack_bf16(o[8 * q + 2] * inv_l + e[8 * q + 2], o[8 * q + 3] * inv_l + e[8 * q + 3]);
-                    w.z = pack_bf16(o[8 * q + 4] * inv_l + e[8 * q + 4], o[8 * q + 5] * inv_l + e[8 * q + 5]);
-                    w.w = pack_bf16(o[8 * q + 6] * inv_l + e[8 * q + 6], o[8 * q + 7] * inv_l + e[8 * q + 7]);
+                    w.x = pack_bf16(o[8 * q + 0] * inv_out + e[8 * q + 0], o[8 * q + 1] * inv_out + e[8 * q + 1]);
+                    w.y = pack_bf16(o[8 * q + 2] * inv_out + e[8 * q + 2], o[8 * q + 3] * inv_out + e[8 * q + 3]);
+                    w.z = pack_bf16(o[8 * q + 4] * inv_out + e[8 * q + 4], o[8 * q + 5] * inv_out + e[8 * q + 5]);
+                    w.w = pack_bf16(o[8 * q + 6] * inv_out + e[8 * q + 6], o[8 * q + 7] * inv_out + e[8 * q + 7]);
                     *reinterpret_cast<uint4*>(smem + Q + hf * kHalf + sw128_offset(r, q)) = w;
                 }
                 fence_async_smem();

@@ -112,6 +112,28 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
                                      float* out_intra, float* out_inter,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* hyb_attn_forward_mixed -- the same pass with a per-(batch, head) weighting of
+ * the two branches: out = a * O_intra + c * O_inter, with (a, c) = mix[b][h]
+ * ([B][H][2] fp32, device memory, 16-byte aligned).  It carries the branch
+ * combinations of the adjacent methods as scalars the caller supplies:
+ * LinVideo ("LinVideo: A Post-Training Framework towards O(n) Attention in
+ * Efficient Video Generation", §2(b) selective transfer) mixes
+ * r * softmax + (1 - r) * linear, i.e. (a, c) = (r, 1 - r); SALAD ("SALAD:
+ * Achieve High-Sparsity Attention via Efficient Linear Attention Tuning for
+ * Video Diffusion Transformer", §2 static-dynamic scaling) scales the linear
+ * branch by a learned static gain g, (1, g), or by a sigmoid-bounded dynamic
+ * factor s = sigmoid(z) computed by the caller, (1, s).  (1, 1) is
+ * hyb_attn_forward.  The state update is unchanged.  c is applied to
+ * W = phi_q^T S_{N-1} before the read (exact: Q (c W) = c O_inter) and a in the
+ * output epilogue.  HYB_ERR_INVALID if mix or out is NULL; otherwise the
+ * arguments and errors of hyb_attn_forward. */
+hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc,
+                                  const void* q, const void* k, const void* v,
+                                  const void* phi_q, const void* phi_k, const void* phi_v,
+                                  const float* gate_logits, const float* beta_logits,
+                                  float* state, int clean_pass, const float* mix, void* out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* hyb_attn_forward_noalloc -- the same pass as hyb_attn_forward for callers
  * that cannot allocate device memory: code running where cudaMalloc is
  * forbidden or unavailable (inside a CUDA graph being captured with a strict

@@ -24,4 +24,5 @@ from .hybrid_layer import (  # noqa: F401
     layer_pass,
     run_frames,
     kvcache_attention,
+    mixed_output,
 )

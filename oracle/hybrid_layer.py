@@ -238,3 +238,17 @@ def kvcache_attention(q, k_frames, v_frames, sm_scale):
     weights = np.exp(scores)
     weights = weights / weights.sum(axis=1, keepdims=True)
     return weights @ v
+
+
+def mixed_output(o_intra, o_inter, a, c):
+    """Weighted combination of the two branches, ``a O_intra + c O_inter``.
+
+    The adjacent methods combine a softmax-type branch with a linear one by a
+    scalar: "LinVideo: A Post-Training Framework towards O(n) Attention in
+    Efficient Video Generation" §2(b) mixes ``r SoftmaxAttn + (1 - r)
+    LinearAttn`` (a = r, c = 1 - r); "SALAD: Achieve High-Sparsity Attention via
+    Efficient Linear Attention Tuning for Video Diffusion Transformer" §2 scales
+    the linear branch by a static gain or a sigmoid-bounded factor (a = 1).
+    a, c: scalars of one (batch, head); o_intra, o_inter: [T, d].
+    """
+    return a * np.asarray(o_intra, dtype=np.float64) + c * np.asarray(o_inter, dtype=np.float64)

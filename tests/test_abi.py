@@ -123,3 +123,14 @@ def test_kvcache_host_validation_rejects_before_launch():
     assert call(kc=FAKE + 8) == G.HYB_ERR_ALIGN
     assert call(ws=None) == G.HYB_ERR_WORKSPACE
     assert call(nbytes=255) == G.HYB_ERR_WORKSPACE
+
+
+def test_mixed_entry_requires_weights():
+    d = G.make_desc(1, 12, 1560, 128)
+    args = [FAKE] * 9
+    assert G.lib.hyb_attn_forward_mixed(ctypes.byref(d), *args, 1, None, FAKE, FAKE, 1 << 40, None) \
+        == G.HYB_ERR_INVALID
+    assert G.lib.hyb_attn_forward_mixed(ctypes.byref(d), *args, 1, FAKE, None, FAKE, 1 << 40, None) \
+        == G.HYB_ERR_INVALID
+    assert G.lib.hyb_attn_forward_mixed(ctypes.byref(d), *args, 1, FAKE + 8, FAKE, FAKE, 1 << 40, None) \
+        == G.HYB_ERR_ALIGN
