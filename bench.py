@@ -50,6 +50,9 @@ def _args():
     p.add_argument("--layer", choices=["hybrid", "kvcache"], default="hybrid",
                    help="hybrid: the ARL2 layer (the reported benchmark); kvcache: the softmax "
                         "baseline with a growing key/value cache on the same stream, for comparison")
+    p.add_argument("--workload", choices=["480p", "long"], default="480p",
+                   help="480p: the reported benchmark; long: the 240-frame B=2 stream (per-frame "
+                        "times over the stream and device memory at frames 1, 60, 120, 240)")
     p.add_argument("--profile-run", action="store_true",
                    help="3 warm-up frames then one frame of the 480p workload; no JSON line "
                         "(a small, fixed launch sequence for ncu captures)")
@@ -464,12 +467,71 @@ def run_kvcache(args):
     return 0
 
 
+def run_long(args):
+    """The long-stream workload (B=2, H=12, 240 frames of 1560 tokens, a pool of
+    8 frames cycled): every frame is timed with CUDA events and device memory is
+    read at frames 1, 60, 120 and 240, once with the state carried through the
+    stream (the literal frame-level rule, whose state leaves the fp32 range
+    mid-stream on these inputs) and once with the state reset every 32 frames
+    (finite data throughout)."""
+    import torch
+    import gated_delta_linear_b200 as G
+    import workloads as W
+
+    w = W.WORKLOADS[4]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pool = []
+    for n in range(w.pool):
+        x = W.pass_inputs(w, n, 0)
+        pool.append([t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)])
+    ph = [p.to(dev) for p in W.feature_maps(w)]
+    out = torch.empty_like(pool[0][0])
+    stream = torch.cuda.current_stream(dev)
+    lines = {}
+    for mode, reset_every in (("state_carried", 0), ("state_reset_every_32", 32)):
+        layer = G.HybridAttention(w.B, w.H, w.T, w.d, torch.bfloat16, *ph, device=dev)
+        for n in range(8):  # warm-up
+            layer.forward(*pool[n % w.pool], 1, out=out)
+        torch.cuda.synchronize(dev)
+        layer.state.zero_()
+        layer.device_status()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.frames + 1)]
+        mem = {}
+        ev[0].record(stream)
+        for n in range(w.frames):
+            if reset_every and n % reset_every == 0:
+                layer.state.zero_()
+            layer.forward(*pool[n % w.pool], 1, out=out)
+            ev[n + 1].record(stream)
+            if n + 1 in (1, 60, 120, 240):
+                torch.cuda.synchronize(dev)
+                free, total = torch.cuda.mem_get_info(dev)
+                mem[str(n + 1)] = total - free
+        torch.cuda.synchronize(dev)
+        us = np.array([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(w.frames)])
+        status = G.hyb_attn_status_string(layer.device_status())
+        lines[mode] = {"us_per_frame_mean": float(us.mean()), "us_first_20": float(us[:20].mean()),
+                       "us_last_20": float(us[-20:].mean()), "cv": float(us.std() / us.mean()),
+                       "device_bytes_in_use_at_frame": mem, "device_status": status}
+    tokens = w.B * w.T
+    line = {"workload": "long_stream_B2_H12_d128_240x1560", "metric": "hybrid-attn layer us per frame over a 240-frame stream",
+            "unit": "us/frame", "value": lines["state_reset_every_32"]["us_per_frame_mean"],
+            "tokens_per_s": tokens / (lines["state_reset_every_32"]["us_per_frame_mean"] / 1e6),
+            "higher_is_better": False, "dtype": "bf16", "data": "synthetic (pool of 8 seeded frames, cycled)",
+            "note": "per-frame CUDA events include the host launch gap between frames", **lines}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         return run_reference(args)
     if args.layer == "kvcache":
         return run_kvcache(args)
+    if args.workload == "long":
+        return run_long(args)
     return run_cuda(args)
 
 
