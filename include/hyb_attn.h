@@ -23,7 +23,8 @@
  *
  * Readings where the pages are silent (all are choices of this library):
  *   - output      out = O_intra + O_inter, rounded once to the I/O dtype
- *                 (the pages do not say how the branches combine);
+ *                 (the pages do not say how the branches combine;
+ *                 hyb_attn_forward_mixed weights the two branches);
  *   - 1x1 maps    x'[o] = sum_i phi[o][i] x[i], i.e. X' = X phi^T; no bias,
  *                 no nonlinearity; the same q, k, v feed both branches;
  *   - K' only     is L2-normalised, as k / sqrt(sum k^2 + l2_eps);
@@ -196,7 +197,8 @@ hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
 /* ---- optional kernel timing (benchmarks) ------------------------------------
  * Process-wide and off by default.  hyb_attn_timing_begin(n) creates 2n CUDA
  * events on the current device; until hyb_attn_timing_end, every kernel that
- * hyb_attn_forward* launches is bracketed by two of them on the call's stream
+ * hyb_attn_forward* or hyb_kvcache_attn_forward (as "intra_frame_attention")
+ * launches is bracketed by two of them on the call's stream
  * (launches beyond n are counted as dropped).  Do not leave timing on while a
  * stream is being captured into a CUDA graph.  hyb_attn_timing_end waits for
  * the recorded events, sums each kernel's launch count and event time into
