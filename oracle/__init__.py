@@ -25,4 +25,5 @@ from .hybrid_layer import (  # noqa: F401
     run_frames,
     kvcache_attention,
     mixed_output,
+    token_level_head_pass,
 )

@@ -252,3 +252,45 @@ def mixed_output(o_intra, o_inter, a, c):
     a, c: scalars of one (batch, head); o_intra, o_inter: [T, d].
     """
     return a * np.asarray(o_intra, dtype=np.float64) + c * np.asarray(o_inter, dtype=np.float64)
+
+
+def token_level_head_pass(q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                          clean_pass, sm_scale=None, l2_eps=1e-6):
+    """The token-level access variant of one pass of one (batch, head) pair.
+
+    ARL2 summary §4 (ablations) compares the layer's frame-level access with a
+    token-level one.  The pages give no formulas for it; the readings taken:
+    on a clean pass the tokens of the frame update the state one after another
+    by the single-token gated delta rule with a per-token forget gate (§2.1
+    calls the forget gate a per-token projection),
+
+        S <- alpha_t S + beta_t k'_t (v'_t^T - k'_t^T S),
+        alpha_t = sigmoid(g_t), beta_t = sigmoid(beta_logit_t),
+
+    and token t reads the state before its own update, O_inter[t] = q'_t S
+    (causal within the frame, the analogue of the frame-level rule's read of
+    S_{N-1}).  A query-only pass updates nothing, so every token reads the
+    frame-start state, as in the frame-level layer.  The intra-frame branch
+    and the combination out = O_intra + O_inter are unchanged.
+    q, k, v: [T, d]; phi_*: [d, d]; gate_logits, beta_logits: [T]; state:
+    [d, d] (not modified).  Returns (out, out_intra, out_inter, new_state).
+    """
+    d = q.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(d)
+    out_intra = intra_frame_attention(q, k, v, sm_scale)
+    q_feat = feature_map(q, phi_q)
+    if not clean_pass:
+        out_inter = inter_frame_read(q_feat, state)
+        return out_intra + out_inter, out_intra, out_inter, state
+    k_unit = l2_normalise_rows(feature_map(k, phi_k), l2_eps)
+    v_feat = feature_map(v, phi_v)
+    alpha = sigmoid(np.asarray(gate_logits, dtype=np.float64))
+    beta = sigmoid(np.asarray(beta_logits, dtype=np.float64))
+    S = np.array(state, dtype=np.float64, copy=True)
+    out_inter = np.empty_like(q_feat)
+    for t in range(q.shape[0]):
+        out_inter[t] = q_feat[t] @ S
+        kt = k_unit[t]
+        S = alpha[t] * S + beta[t] * np.outer(kt, v_feat[t] - kt @ S)
+    return out_intra + out_inter, out_intra, out_inter, S
