@@ -107,7 +107,37 @@ def pin_product_form_of_the_recurrence():
             np.testing.assert_allclose(S, St, rtol=1e-10, atol=1e-10)
 
 
-PINS = [pin_one_token_is_the_frame_level_rule, pin_single_token_stores_its_value,
+def pin_chunked_triangular_solve_form():
+    # The same recurrence in chunks of C tokens, as a kernel would compute it.
+    # With gamma_t = alpha_1 ... alpha_t and the normalised state S^_t = S_t / gamma_t,
+    #   S^_t = S^_{t-1} + k_t u_t^T,  u_t = c_t v'_t - b_t S^_{t-1}^T k_t,
+    #   b_t = beta_t / alpha_t, c_t = beta_t / gamma_t,
+    # so per chunk (I + diag(b) tril(K K^T, -1)) U = diag(c) V - diag(b) K S^_0,
+    # S^_C = S^_0 + K^T U, and token t reads gamma_{t-1} (q_t S^_0 + sum_{r<t} (q_t . k_r) u_r).
+    q, k, v, phi, g, bl, S0 = _inputs(7, T=11)
+    _, _, oe, S = O.token_level_head_pass(q, k, v, *phi, g, bl, S0, True)
+    kf = k @ phi[1].T
+    ku = kf / np.sqrt((kf ** 2).sum(axis=1, keepdims=True) + 1e-6)
+    vf, qf = v @ phi[2].T, q @ phi[0].T
+    al, be = 1 / (1 + np.exp(-g)), 1 / (1 + np.exp(-bl))
+    Sc = S0.copy()
+    reads = np.empty_like(oe)
+    C = 4
+    for c0 in range(0, 11, C):
+        sl = slice(c0, min(11, c0 + C))
+        K, V, Q, a, bt = ku[sl], vf[sl], qf[sl], al[sl], be[sl]
+        gam = np.cumprod(a)
+        gam_prev = np.concatenate([[1.0], gam[:-1]])
+        b, cc = bt / a, bt / gam
+        L = np.eye(len(a)) + np.diag(b) @ np.tril(K @ K.T, -1)
+        U = np.linalg.solve(L, np.diag(cc) @ V - np.diag(b) @ K @ Sc)
+        reads[sl] = gam_prev[:, None] * (Q @ Sc + np.tril(Q @ K.T, -1) @ U)
+        Sc = gam[-1] * (Sc + K.T @ U)
+    np.testing.assert_allclose(oe, reads, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(S, Sc, rtol=1e-9, atol=1e-9)
+
+
+PINS = [pin_chunked_triangular_solve_form, pin_one_token_is_the_frame_level_rule, pin_single_token_stores_its_value,
         pin_orthonormal_keys_match_the_frame_level_update, pin_query_only_pass_is_the_frame_level_pass,
         pin_each_step_is_non_expansive, pin_product_form_of_the_recurrence]
 
