@@ -169,19 +169,49 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// Encoded tensor maps of recent calls, per host thread: a frame loop passes
+// the same buffers again and again, so most calls find every map here and
+// skip the driver's encoder.  The key is everything the encoding depends on.
+struct MapKey {
+    const void* base;
+    uint64_t d0, d1, d2, s1, s2;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && s1 == o.s1 && s2 == o.s2;
+    }
+};
+struct MapCache {
+    static constexpr int kEntries = 32;
+    MapKey key[kEntries];
+    CUtensorMap map[kEntries];
+    int used = 0, next = 0;
+};
+thread_local MapCache t_maps;
+
 // 3-D bf16 tensor map with 64 x 128 x 1 boxes and 128-byte swizzle:
 // dims {d0 (contiguous), d1, d2}, byte strides s1, s2 of dims 1 and 2.
 bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
            uint64_t s2) {
+    const MapKey k = {base, d0, d1, d2, s1, s2};
+    MapCache& c = t_maps;
+    for (int i = 0; i < c.used; ++i)
+        if (c.key[i] == k) {
+            *m = c.map[i];
+            return true;
+        }
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {s1, s2};
     cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    const int slot = c.used < MapCache::kEntries ? c.used++ : c.next++ % MapCache::kEntries;
+    c.key[slot] = k;
+    c.map[slot] = *m;
+    return true;
 }
 
 cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
@@ -256,11 +286,13 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
-                        const void* phi_q, const void* phi_k, const void* phi_v,
-                        const float* gate_logits, const float* beta_logits, float* state,
-                        int clean_pass, void* out, float* out_intra, float* out_inter,
-                        void* workspace, size_t workspace_bytes, void* stream, const float* mix = nullptr) {
+// Checks every argument of a pass and fills the kernels' argument block;
+// enqueues nothing, so an error here leaves the stream untouched.
+hyb_status pass_args(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                     const void* phi_q, const void* phi_k, const void* phi_v, const float* gate_logits,
+                     const float* beta_logits, float* state, int clean_pass, void* out, float* out_intra,
+                     float* out_inter, void* workspace, size_t workspace_bytes, const float* mix,
+                     LayerArgs* args, Plan* plan) {
     Plan p;
     hyb_status s = make_plan(desc, &p);
     if (s != HYB_OK) return s;
@@ -308,7 +340,12 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.partials = (float*)(ws + p.off_part);
     a.nsplit = p.nsplit;
     a.split_tokens = p.split_tokens;
+    *args = a;
+    *plan = p;
+    return HYB_OK;
+}
 
+hyb_status launch_pass(const LayerArgs& a, const Plan& p, int clean_pass, void* stream) {
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     if (p.bf16)
@@ -316,6 +353,19 @@ hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     else
         e = launch_simt<32, float>(a, clean_pass, st);
     return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
+hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                        const void* phi_q, const void* phi_k, const void* phi_v,
+                        const float* gate_logits, const float* beta_logits, float* state,
+                        int clean_pass, void* out, float* out_intra, float* out_inter,
+                        void* workspace, size_t workspace_bytes, void* stream, const float* mix = nullptr) {
+    LayerArgs a;
+    Plan p;
+    hyb_status s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass,
+                             out, out_intra, out_inter, workspace, workspace_bytes, mix, &a, &p);
+    if (s != HYB_OK) return s;
+    return launch_pass(a, p, clean_pass, stream);
 }
 
 // Softmax attention of one frame's queries over a KV cache (the baseline the
@@ -568,12 +618,20 @@ extern "C" hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc, const 
     hyb_status s = make_plan(desc, &p);
     if (s != HYB_OK) return s;
     if (p.total > (size_t)HYB_NOALLOC_SCRATCH_BYTES) return HYB_ERR_WORKSPACE;
+    // every argument is checked before any CUDA call (with a stand-in for the
+    // scratch address, which is looked up only afterwards)
+    LayerArgs a;
+    s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out, nullptr,
+                  nullptr, (void*)(uintptr_t)256, HYB_NOALLOC_SCRATCH_BYTES, nullptr, &a, &p);
+    if (s != HYB_OK) return s;
     cudaError_t e;
     void* scratch = noalloc_scratch(&e);
     if (!scratch) return HYB_ERR_CUDA;
+    s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out, nullptr,
+                  nullptr, scratch, HYB_NOALLOC_SCRATCH_BYTES, nullptr, &a, &p);
+    if (s != HYB_OK) return s;
     // the status word accumulates flags: start every call from zero
     if (cudaMemsetAsync(scratch, 0, sizeof(unsigned), (cudaStream_t)stream) != cudaSuccess)
         return HYB_ERR_CUDA;
-    return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
-                        clean_pass, out, nullptr, nullptr, scratch, HYB_NOALLOC_SCRATCH_BYTES, stream);
+    return launch_pass(a, p, clean_pass, stream);
 }

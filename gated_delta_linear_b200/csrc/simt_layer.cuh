@@ -55,10 +55,9 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
     const size_t bh = (size_t)b * a.H + h;
     if constexpr (kSplitOut) {
         // tensor path, launched as a programmatic dependent: wait until the
-        // previous kernel (which may write the state) has completed, then let the
-        // attention kernel start; it reads W only after this grid completes
+        // previous kernel (which may write the state) has completed before
+        // reading S_{N-1}
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     }
     // all loads of a thread are issued before any shared-memory store: the
     // stores go through generic pointers, which would otherwise serialise them
@@ -82,6 +81,13 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
         for (int u = 0; u < NP; ++u) Ph[tid + u * kThreads] = pv[u];
     }
     __syncthreads();
+    if constexpr (kSplitOut) {
+        // S_{N-1} is in shared memory: only now may the attention kernel start,
+        // and through it the delta update that overwrites the state in place
+        // (it is launched once every attention CTA has started).  The attention
+        // kernel reads W only after this grid has completed.
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     // each warp owns rows r0..r0+RW-1 of W; each lane NC consecutive columns
     const int r0 = RW * warp;
     float acc[RW][NC];
