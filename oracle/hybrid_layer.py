@@ -269,7 +269,12 @@ def token_level_head_pass(q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits
 
     and token t reads the state before its own update, O_inter[t] = q'_t S
     (causal within the frame, the analogue of the frame-level rule's read of
-    S_{N-1}).  A query-only pass updates nothing, so every token reads the
+    S_{N-1}).  The residual v'_t - k'_t^T S is taken against the undecayed
+    state, exactly as in the frame-level rule of §2.1 (so a one-token frame
+    gives the same update under both accesses).  This is a reading, not the
+    form of "Gated Delta Networks", whose rule S <- alpha S (I - beta k k^T) +
+    beta v k^T decays the state inside the residual; the two differ whenever
+    alpha_t < 1.  A query-only pass updates nothing, so every token reads the
     frame-start state, as in the frame-level layer.  The intra-frame branch
     and the combination out = O_intra + O_inter are unchanged.
     q, k, v: [T, d]; phi_*: [d, d]; gate_logits, beta_logits: [T]; state:

@@ -107,37 +107,71 @@ def pin_product_form_of_the_recurrence():
             np.testing.assert_allclose(S, St, rtol=1e-10, atol=1e-10)
 
 
+def _chunked_pass(q, k, v, phi, g, bl, S0, C, dtype):
+    """The token-level recurrence in chunks of C tokens, as a kernel computes it,
+    with only relative decays (every factor exp(Lambda_a - Lambda_b) <= 1,
+    Lambda_t = sum_{r <= t} log alpha_r; nothing is divided by a gate).
+    Inside a chunk that starts from state S, with u_t the row beta_t (v'_t - k'_t S_{t-1}):
+      (I + L) U = diag(beta) V - diag(beta * gprev) K S,
+      L[t, s] = beta_t exp(Lambda_{t-1} - Lambda_s) (k_t . k_s)      for s < t,
+      gprev_t = exp(Lambda_{t-1})  (the decay from the chunk start to token t's read),
+      read_t  = gprev_t q_t S + sum_{s<t} exp(Lambda_{t-1} - Lambda_s) (q_t . k_s) u_s,
+      S_end   = exp(Lambda_{C-1}) S + sum_s exp(Lambda_{C-1} - Lambda_s) k_s u_s."""
+    f = lambda x: np.asarray(x, dtype=dtype)
+    kf = k @ phi[1].T
+    ku = f(kf / np.sqrt((kf ** 2).sum(axis=1, keepdims=True) + 1e-6))
+    vf, qf = f(v @ phi[2].T), f(q @ phi[0].T)
+    logal = f(-np.logaddexp(0.0, -np.asarray(g, dtype=np.float64)))  # log sigmoid(g), no overflow
+    be = f(1 / (1 + np.exp(-np.asarray(bl, dtype=np.float64))))
+    T = q.shape[0]
+    Sc = f(S0)
+    reads = np.empty((T, S0.shape[1]), dtype=dtype)
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(T, c0 + C))
+        K, V, Q, la, bt = ku[sl], vf[sl], qf[sl], logal[sl], be[sl]
+        n = len(la)
+        Lam = np.cumsum(la)                                   # Lambda_t within the chunk
+        Lprev = np.concatenate([np.zeros(1, dtype=dtype), Lam[:-1]])
+        dec = np.exp(np.minimum(Lprev[:, None] - Lam[None, :], 0.0))  # exp(Lambda_{t-1} - Lambda_s)
+        strict = np.tril(np.ones((n, n), dtype=dtype), -1)
+        A = strict * dec * (K @ K.T)
+        gprev = np.exp(Lprev)
+        U = np.linalg.solve(np.eye(n, dtype=dtype) + bt[:, None] * A,
+                            bt[:, None] * V - (bt * gprev)[:, None] * (K @ Sc))
+        reads[sl] = gprev[:, None] * (Q @ Sc) + (strict * dec * (Q @ K.T)) @ U
+        Sc = np.exp(Lam[-1]) * Sc + K.T @ (np.exp(Lam[-1] - Lam)[:, None] * U)
+    return reads, Sc
+
+
 def pin_chunked_triangular_solve_form():
-    # The same recurrence in chunks of C tokens, as a kernel would compute it.
-    # With gamma_t = alpha_1 ... alpha_t and the normalised state S^_t = S_t / gamma_t,
-    #   S^_t = S^_{t-1} + k_t u_t^T,  u_t = c_t v'_t - b_t S^_{t-1}^T k_t,
-    #   b_t = beta_t / alpha_t, c_t = beta_t / gamma_t,
-    # so per chunk (I + diag(b) tril(K K^T, -1)) U = diag(c) V - diag(b) K S^_0,
-    # S^_C = S^_0 + K^T U, and token t reads gamma_{t-1} (q_t S^_0 + sum_{r<t} (q_t . k_r) u_r).
+    # float64, chunks of 4 over 11 tokens: the chunked form equals the token loop
     q, k, v, phi, g, bl, S0 = _inputs(7, T=11)
     _, _, oe, S = O.token_level_head_pass(q, k, v, *phi, g, bl, S0, True)
-    kf = k @ phi[1].T
-    ku = kf / np.sqrt((kf ** 2).sum(axis=1, keepdims=True) + 1e-6)
-    vf, qf = v @ phi[2].T, q @ phi[0].T
-    al, be = 1 / (1 + np.exp(-g)), 1 / (1 + np.exp(-bl))
-    Sc = S0.copy()
-    reads = np.empty_like(oe)
-    C = 4
-    for c0 in range(0, 11, C):
-        sl = slice(c0, min(11, c0 + C))
-        K, V, Q, a, bt = ku[sl], vf[sl], qf[sl], al[sl], be[sl]
-        gam = np.cumprod(a)
-        gam_prev = np.concatenate([[1.0], gam[:-1]])
-        b, cc = bt / a, bt / gam
-        L = np.eye(len(a)) + np.diag(b) @ np.tril(K @ K.T, -1)
-        U = np.linalg.solve(L, np.diag(cc) @ V - np.diag(b) @ K @ Sc)
-        reads[sl] = gam_prev[:, None] * (Q @ Sc + np.tril(Q @ K.T, -1) @ U)
-        Sc = gam[-1] * (Sc + K.T @ U)
+    reads, Sc = _chunked_pass(q, k, v, phi, g, bl, S0, 4, np.float64)
     np.testing.assert_allclose(oe, reads, rtol=1e-9, atol=1e-9)
     np.testing.assert_allclose(S, Sc, rtol=1e-9, atol=1e-9)
 
 
-PINS = [pin_chunked_triangular_solve_form, pin_one_token_is_the_frame_level_rule, pin_single_token_stores_its_value,
+def pin_chunked_form_in_fp32_with_strong_forgetting():
+    # fp32, chunks of 64 over 150 tokens (a ragged last chunk), gate logits down to
+    # -6 (alpha ~ 2.5e-3): the relative-decay form stays finite and accurate
+    rng = np.random.default_rng(8)
+    T, d = 150, 32
+    q, k, v = (rng.standard_normal((T, d)) for _ in range(3))
+    phi = [np.eye(d) + 0.02 * rng.standard_normal((d, d)) for _ in range(3)]
+    g = rng.uniform(-6.0, 3.0, T)
+    g[::7] = -6.0
+    bl = rng.standard_normal(T)
+    S0 = rng.standard_normal((d, d))
+    _, _, oe, S = O.token_level_head_pass(q, k, v, *phi, g, bl, S0, True)
+    reads, Sc = _chunked_pass(q, k, v, phi, g, bl, S0, 64, np.float32)
+    assert np.isfinite(reads).all() and np.isfinite(Sc).all()
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert rel(reads.astype(np.float64), oe) < 1e-4, rel(reads.astype(np.float64), oe)
+    assert rel(Sc.astype(np.float64), S) < 1e-4, rel(Sc.astype(np.float64), S)
+
+
+PINS = [pin_chunked_triangular_solve_form, pin_chunked_form_in_fp32_with_strong_forgetting, pin_one_token_is_the_frame_level_rule, pin_single_token_stores_its_value,
         pin_orthonormal_keys_match_the_frame_level_update, pin_query_only_pass_is_the_frame_level_pass,
         pin_each_step_is_non_expansive, pin_product_form_of_the_recurrence]
 
