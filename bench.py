@@ -37,6 +37,13 @@ sys.path.insert(0, ROOT)
 METRIC = "hybrid-attn layer tokens/s (21-frame 480p forward, 1 B200)"
 UNIT = "tokens/s"
 WORKLOAD_ID = 1
+WORKLOAD_IDS = {"480p": 1, "stream14b": 2, "720p": 3}
+METRICS = {
+    "480p": METRIC,
+    "stream14b": "hybrid-attn layer tokens/s (Wan-14B streaming step: one 1560-token frame, "
+                 "4 query-only + 1 clean pass on a prebuilt state, 1 B200)",
+    "720p": "hybrid-attn layer tokens/s (21-frame 720p forward, H40, 1 B200)",
+}
 
 
 def _args():
@@ -50,9 +57,12 @@ def _args():
     p.add_argument("--layer", choices=["hybrid", "kvcache"], default="hybrid",
                    help="hybrid: the ARL2 layer (the reported benchmark); kvcache: the softmax "
                         "baseline with a growing key/value cache on the same stream, for comparison")
-    p.add_argument("--workload", choices=["480p", "long"], default="480p",
-                   help="480p: the reported benchmark; long: the 240-frame B=2 stream (per-frame "
-                        "times over the stream and device memory at frames 1, 60, 120, 240)")
+    p.add_argument("--workload", choices=["480p", "720p", "stream14b", "long"], default="480p",
+                   help="480p: the reported benchmark (21 frames of 1560 tokens, H12); 720p: 21 frames "
+                        "of 3600 tokens, H40; stream14b: one frame of the Wan-14B shape (H40) as 4 "
+                        "query-only passes and a clean pass on a state built from 20 prior frames "
+                        "(per-frame latency); long: the 240-frame B=2 stream (per-frame times over "
+                        "the stream and device memory at frames 1, 60, 120, 240)")
     p.add_argument("--profile-run", action="store_true",
                    help="3 warm-up frames then one frame of the 480p workload; no JSON line "
                         "(a small, fixed launch sequence for ncu captures)")
@@ -93,6 +103,45 @@ def oracle_frames(w, max_seconds, max_frames=None):
         spent += time.perf_counter() - t0
         done += 1
     return done, spent
+
+
+def _inputs_note(w):
+    nbytes = 3 * w.frames * len(w.passes) * w.B * w.T * w.H * w.d * 2
+    big = nbytes > 126e6
+    return (f"all {w.frames * len(w.passes)} passes' q/k/v resident in HBM ({nbytes / 1e6:.0f} MB"
+            + (" > 126 MB L2); no L2 flush needed" if big else
+               " < 126 MB L2: consecutive steps may hit in L2 on their inputs)"))
+
+
+def oracle_head_sample(w, max_seconds):
+    """The float64 oracle on a bounded sample of a large workload: whole
+    (frame, pass, head) units of its first frame, one head at a time, until
+    max_seconds; scaled to the metric (each unit stands for T / H of the frame's
+    tokens and 1 / passes of its passes)."""
+    import torch
+    import oracle
+    import workloads as W
+    phi = [p.to(torch.float64).numpy() for p in W.feature_maps(w)]
+    S = W.zero_state(w)
+    units, spent = 0, 0.0
+    for p, clean in enumerate(w.passes):
+        x = W.pass_inputs(w, 0, p).as_f64()
+        for b in range(w.B):
+            for h in range(w.H):
+                t0 = time.perf_counter()
+                oracle.layer_pass(*x[:3], *phi, *x[3:], S, clean, heads=[(b, h)])
+                spent += time.perf_counter() - t0
+                units += 1
+                if spent >= max_seconds:
+                    break
+            if spent >= max_seconds:
+                break
+        if spent >= max_seconds:
+            break
+    per_unit = w.T / w.H / len(w.passes)
+    return {"value": units * per_unit / spent, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"{units} (pass, head) units of frame 0 ({w.H} heads x {len(w.passes)} passes per frame), "
+                      f"{spent:.1f} s of float64 NumPy, scaled by T/H/passes per unit"}
 
 
 def oracle_one_thread(w, max_seconds):
@@ -256,10 +305,14 @@ def run_cuda(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w = W.WORKLOADS[WORKLOAD_ID]
+    wid = WORKLOAD_IDS[args.workload]
+    w = W.WORKLOADS[wid]
     phi = W.feature_maps(w)
     layer = G.HybridAttention(w.B, w.H, w.T, w.d, w.torch_dtype, *phi, device=dev)
-    host = [W.pass_inputs(w, n, 0) for n in range(w.frames)]
+    # every pass of every frame, in order (480p / 720p: one clean pass per frame;
+    # the streaming step: 4 query-only passes and a clean pass of one frame)
+    cleans = [int(c) for _ in range(w.frames) for c in w.passes]
+    host = [W.pass_inputs(w, n, p) for n in range(w.frames) for p in range(len(w.passes))]
     frames = [[t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)] for x in host]
     outs = [torch.empty_like(f[0]) for f in frames]
     stream = torch.cuda.current_stream(dev)
@@ -268,15 +321,24 @@ def run_cuda(args):
     phis = [p.data_ptr() for p in layer.phi]
     state_ptr, ws_ptr = layer.state.data_ptr(), layer.workspace.data_ptr()
     calls = [[f[0].data_ptr(), f[1].data_ptr(), f[2].data_ptr(), *phis, f[3].data_ptr(),
-              f[4].data_ptr(), state_ptr, 1, o.data_ptr(), ws_ptr, wsb, sptr]
-             for f, o in zip(frames, outs)]
+              f[4].data_ptr(), state_ptr, c, o.data_ptr(), ws_ptr, wsb, sptr]
+             for f, o, c in zip(frames, outs, cleans)]
     desc = layer.desc
     fwd = G.lib.hyb_attn_forward
     import ctypes
     dref = ctypes.byref(desc)
+    # initial state of the step: S_0 = 0, or (streaming step) the state the layer
+    # itself builds from the workload's prior frames, kept and restored each step
+    state0 = torch.zeros_like(layer.state)
+    if w.prior_frames:
+        for j in range(w.prior_frames):
+            x = W.prior_frame_inputs(w, j)
+            layer.forward(*[t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)], 1)
+        torch.cuda.synchronize(dev)
+        state0.copy_(layer.state)
 
     def step():
-        layer.state.zero_()
+        layer.state.copy_(state0)
         for c in calls:
             st = fwd(dref, *c)
             if st != G.HYB_OK:
@@ -334,7 +396,8 @@ def run_cuda(args):
     burst, sustained, hbm, src = _peaks()
     achieved = attention_flops(w) / avg_attn_s / 1e12
     frame_s = ms / 1e3 / args.steps / w.frames
-    layer_tf = layer_flops(w) / frame_s / 1e12
+    frame_flops = sum(layer_flops(w, bool(c)) for c in w.passes)   # every pass of one frame
+    layer_tf = frame_flops / frame_s / 1e12
     roofline = {"kernel": "intra_frame_attention", "bound": "tensor", "achieved": achieved,
                 "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
                 "peak_source": f"{src} bf16_tflops (burst: each launch is timed alone between its own "
@@ -343,7 +406,7 @@ def run_cuda(args):
                 "avg_launch_us": avg_attn_s * 1e6,
                 "flops_per_launch": attention_flops(w),
                 "dominant_kernel_by_time": name,
-                "layer": {"flops_per_frame": layer_flops(w), "us_per_frame": frame_s * 1e6,
+                "layer": {"flops_per_frame": frame_flops, "us_per_frame": frame_s * 1e6,
                           "achieved": layer_tf, "frac": layer_tf / burst,
                           "timed_region": "A (the reported value: no per-kernel events)"},
                 "kernel_ms": {k: v[1] for k, v in per_kernel.items()},
@@ -365,7 +428,7 @@ def run_cuda(args):
     d2h = sum(o.numel() * o.element_size() for o in hout)
 
     def e2e_step():
-        layer.state.zero_()
+        layer.state.copy_(state0)
         for f, hf, c, o, ho in zip(frames, pin, calls, outs, hout):
             for dst, src_ in zip(f, hf):
                 dst.copy_(src_, non_blocking=True)
@@ -389,11 +452,14 @@ def run_cuda(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, s = oracle_frames(w, args.cpu_baseline_seconds)
-        cpu = {"value": w.B * w.T * n / s, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-               "sample": f"first {n} of {w.frames} frames (all {w.H} heads, state carried), "
-                         f"{s:.1f} s of float64 NumPy"}
-        cpu["one_thread"] = oracle_one_thread(w, args.cpu_baseline_seconds / 2)
+        if args.workload == "480p":
+            n, s = oracle_frames(w, args.cpu_baseline_seconds)
+            cpu = {"value": w.B * w.T * n / s, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                   "sample": f"first {n} of {w.frames} frames (all {w.H} heads, state carried), "
+                             f"{s:.1f} s of float64 NumPy"}
+            cpu["one_thread"] = oracle_one_thread(w, args.cpu_baseline_seconds / 2)
+        else:
+            cpu = oracle_head_sample(w, args.cpu_baseline_seconds)
 
     if world > 1:
         dist.barrier()
@@ -401,12 +467,12 @@ def run_cuda(args):
     if rank != 0:
         return 0
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRICS[args.workload], "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
         "us_per_frame": 1e3 * ms / args.steps / w.frames,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded normals, video-DiT shapes)",
-        "config": _config(w),
+        "config": _config(w, {"inputs": _inputs_note(w)}),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -496,11 +562,14 @@ def run_kvcache(args):
 
 def run_long(args):
     """The long-stream workload (B=2, H=12, 240 frames of 1560 tokens, a pool of
-    8 frames cycled): every frame is timed with CUDA events and device memory is
-    read at frames 1, 60, 120 and 240, once with the state carried through the
-    stream (the literal frame-level rule, whose state leaves the fp32 range
-    mid-stream on these inputs) and once with the state reset every 32 frames
-    (finite data throughout)."""
+    8 frames cycled), once with the state carried through the stream (the literal
+    frame-level rule, whose state leaves the fp32 range mid-stream on these
+    inputs) and once with the state reset every 32 frames (finite data
+    throughout).  Device memory is read at frames 1, 60, 120 and 240 in a pass
+    of its own (each reading synchronises); throughput is timed in a second pass
+    with no host synchronisation, as windows of 20 frames enqueued back to back,
+    each window between two CUDA events, so host gaps between frames do not
+    enter the per-frame times."""
     import torch
     import gated_delta_linear_b200 as G
     import workloads as W
@@ -515,38 +584,59 @@ def run_long(args):
     ph = [p.to(dev) for p in W.feature_maps(w)]
     out = torch.empty_like(pool[0][0])
     stream = torch.cuda.current_stream(dev)
+    window = 20
     lines = {}
     for mode, reset_every in (("state_carried", 0), ("state_reset_every_32", 32)):
         layer = G.HybridAttention(w.B, w.H, w.T, w.d, torch.bfloat16, *ph, device=dev)
         for n in range(8):  # warm-up
             layer.forward(*pool[n % w.pool], 1, out=out)
         torch.cuda.synchronize(dev)
-        layer.state.zero_()
-        layer.device_status()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.frames + 1)]
+
+        def stream_frames(on_frame=None):
+            layer.state.zero_()
+            for n in range(w.frames):
+                if reset_every and n % reset_every == 0:
+                    layer.state.zero_()
+                layer.forward(*pool[n % w.pool], 1, out=out)
+                if on_frame:
+                    on_frame(n)
+
+        # pass 1: device memory in use at frames 1, 60, 120, 240
         mem = {}
-        ev[0].record(stream)
-        for n in range(w.frames):
-            if reset_every and n % reset_every == 0:
-                layer.state.zero_()
-            layer.forward(*pool[n % w.pool], 1, out=out)
-            ev[n + 1].record(stream)
+
+        def read_mem(n):
             if n + 1 in (1, 60, 120, 240):
                 torch.cuda.synchronize(dev)
                 free, total = torch.cuda.mem_get_info(dev)
                 mem[str(n + 1)] = total - free
+
+        stream_frames(read_mem)
         torch.cuda.synchronize(dev)
-        us = np.array([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(w.frames)])
+        layer.device_status()
+        # pass 2: windows of `window` frames between events, no host synchronisation
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.frames // window + 1)]
+
+        def mark(n):
+            if (n + 1) % window == 0:
+                ev[(n + 1) // window].record(stream)
+
+        ev[0].record(stream)
+        stream_frames(mark)
+        torch.cuda.synchronize(dev)
+        us = np.array([ev[i].elapsed_time(ev[i + 1]) * 1e3 / window for i in range(len(ev) - 1)])
         status = G.hyb_attn_status_string(layer.device_status())
-        lines[mode] = {"us_per_frame_mean": float(us.mean()), "us_first_20": float(us[:20].mean()),
-                       "us_last_20": float(us[-20:].mean()), "cv": float(us.std() / us.mean()),
+        lines[mode] = {"us_per_frame_mean": float(us.mean()), "us_per_frame_first_window": float(us[0]),
+                       "us_per_frame_last_window": float(us[-1]), "cv_over_windows": float(us.std() / us.mean()),
+                       "windows": len(us), "frames_per_window": window,
                        "device_bytes_in_use_at_frame": mem, "device_status": status}
     tokens = w.B * w.T
     line = {"workload": "long_stream_B2_H12_d128_240x1560", "metric": "hybrid-attn layer us per frame over a 240-frame stream",
             "unit": "us/frame", "value": lines["state_reset_every_32"]["us_per_frame_mean"],
             "tokens_per_s": tokens / (lines["state_reset_every_32"]["us_per_frame_mean"] / 1e6),
             "higher_is_better": False, "dtype": "bf16", "data": "synthetic (pool of 8 seeded frames, cycled)",
-            "note": "per-frame CUDA events include the host launch gap between frames", **lines}
+            "note": "windows of 20 frames enqueued back to back, each between two CUDA events (no host "
+                    "synchronisation inside a window); the state resets inside the timed windows are "
+                    "included in the reset-every-32 figures", **lines}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -559,6 +649,9 @@ def main():
         return run_kvcache(args)
     if args.workload == "long":
         return run_long(args)
+    if args.workload != "480p" and args.gpus > 1:
+        print(json.dumps({"error": "--workload other than 480p runs on one GPU"}))
+        return 2
     return run_cuda(args)
 
 

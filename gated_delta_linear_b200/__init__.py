@@ -33,9 +33,13 @@ from ._binding import (  # noqa: F401
     hyb_kvcache_attn_forward,
     hyb_attn_forward_mixed,
     HybridAttention,
+    TokenLevelAttention,
+    hyb_attn_forward_token_level,
+    hyb_attn_token_level_workspace_bytes,
     KVCacheAttention,
     HybAttnTiming,
     HYB_NUM_KERNELS,
+    hyb_attn_set_fault_test,
     hyb_attn_timing_begin,
     hyb_attn_timing_end,
     hyb_attn_kernel_name,

@@ -35,7 +35,7 @@ class HybAttnDesc(ctypes.Structure):
     ]
 
 
-HYB_NUM_KERNELS = 4
+HYB_NUM_KERNELS = 7
 
 
 class HybAttnTiming(ctypes.Structure):
@@ -62,10 +62,16 @@ def _load():
     L.hyb_attn_forward_noalloc.restype = i
     L.hyb_attn_forward_mixed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.hyb_attn_forward_mixed.restype = i
+    L.hyb_attn_token_level_workspace_bytes.argtypes = [dp]
+    L.hyb_attn_token_level_workspace_bytes.restype = sz
+    L.hyb_attn_forward_token_level.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
+    L.hyb_attn_forward_token_level.restype = i
     L.hyb_kvcache_attn_forward.argtypes = [dp, vp, vp, vp, vp, vp, i, i, vp, vp, sz, vp]
     L.hyb_kvcache_attn_forward.restype = i
     L.hyb_attn_get_device_status.argtypes = [vp, vp]
     L.hyb_attn_get_device_status.restype = i
+    L.hyb_attn_set_fault_test.argtypes = [i, ctypes.c_uint]
+    L.hyb_attn_set_fault_test.restype = i
     L.hyb_attn_timing_begin.argtypes = [i]
     L.hyb_attn_timing_begin.restype = i
     L.hyb_attn_timing_end.argtypes = [ctypes.POINTER(HybAttnTiming)]
@@ -140,6 +146,20 @@ def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, be
                                         _stream(stream))
 
 
+def hyb_attn_token_level_workspace_bytes(desc: HybAttnDesc) -> int:
+    return lib.hyb_attn_token_level_workspace_bytes(ctypes.byref(desc))
+
+
+def hyb_attn_forward_token_level(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                                 clean_pass, out, workspace, workspace_bytes=None, stream=None) -> int:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_attn_forward_token_level(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(phi_q),
+                                            _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits), _ptr(beta_logits),
+                                            _ptr(state), int(clean_pass), _ptr(out), _ptr(workspace),
+                                            workspace_bytes, _stream(stream))
+
+
 def hyb_attn_forward_mixed(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
                            clean_pass, mix, out, workspace, workspace_bytes=None, stream=None) -> int:
     if workspace_bytes is None:
@@ -165,6 +185,12 @@ def hyb_attn_get_device_status(workspace, stream=None) -> int:
 
 def hyb_attn_status_string(status: int) -> str:
     return lib.hyb_attn_status_string(int(status)).decode()
+
+
+def hyb_attn_set_fault_test(skip_v_loads: int, wait_limit_us: int) -> int:
+    """Test hook (off by default): shorten the attention kernel's bounded waits
+    and/or switch off its value-tile loads so that a wait expires."""
+    return lib.hyb_attn_set_fault_test(int(skip_v_loads), int(wait_limit_us))
 
 
 def hyb_attn_timing_begin(max_launches: int) -> int:
@@ -241,6 +267,30 @@ class HybridAttention:
 
     def device_status(self, stream=None) -> int:
         return hyb_attn_get_device_status(self.workspace, stream)
+
+
+class TokenLevelAttention(HybridAttention):
+    """The token-level access variant of the layer (tokens update the state one
+    after another on a clean pass); the same buffers as HybridAttention with the
+    larger workspace hyb_attn_token_level_workspace_bytes asks for."""
+
+    def __init__(self, B, H, T, d, dtype, phi_q, phi_k, phi_v, device="cuda", sm_scale=0.0, l2_eps=1e-6):
+        import torch
+        super().__init__(B, H, T, d, dtype, phi_q, phi_k, phi_v, device, sm_scale, l2_eps)
+        nbytes = hyb_attn_token_level_workspace_bytes(self.desc)
+        if nbytes == 0:
+            raise HybAttnError(HYB_ERR_UNSUPPORTED, "hyb_attn_token_level_workspace_bytes")
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+
+    def forward(self, q, k, v, gate_logits, beta_logits, clean_pass, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        st = hyb_attn_forward_token_level(self.desc, q, k, v, *self.phi, gate_logits, beta_logits, self.state,
+                                          clean_pass, out, self.workspace, stream=stream)
+        if st != HYB_OK:
+            raise HybAttnError(st, "hyb_attn_forward_token_level")
+        return out
 
 
 class KVCacheAttention:

@@ -43,6 +43,12 @@ struct LayerArgs {
     float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
     int nsplit;
     int split_tokens;
+    // token-level access: the inter-frame read computed by the token-level kernels,
+    // fp32 [B][T][H][D]; the attention kernels add it instead of Q W (NULL: Q W)
+    const float* oi_ext;
+    // bounded device waits give up after wait_ns (2 s unless a fault test shortens it)
+    unsigned long long wait_ns;
+    int dbg_skip_v;            // fault test only: the attention kernel's V producer issues nothing
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -14,6 +14,8 @@
 #include "common.cuh"
 #include "simt_layer.cuh"
 #include "tc_kernels.cuh"
+#include "tc_attention.cuh"
+#include "token_level.cuh"
 
 namespace {
 
@@ -52,6 +54,12 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     const int BH = d->B * d->H;
     const int ntiles = (d->T + kUpdateTile - 1) / kUpdateTile;
     int want = bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH;
+    if (bf16) {
+        // the update runs beside the attention kernel (two query tiles per CTA):
+        // size its clusters to the SMs that grid leaves free, when it leaves some
+        const long attn_ctas = (long)((ntiles + 1) / 2) * BH;
+        if (attn_ctas < kNumSMs && (kNumSMs - attn_ctas) / BH >= 2) want = (int)((kNumSMs - attn_ctas) / BH);
+    }
     if (bf16 && want > tc::kMaxClusterRanks) want = tc::kMaxClusterRanks;
     if (want > ntiles) want = ntiles;
     if (want < 1) want = 1;
@@ -69,7 +77,7 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
 }
 
 // ---- optional kernel timing -------------------------------------------------
-enum { K_PREP = 0, K_ATTN = 1, K_UPDATE = 2, K_APPLY = 3 };
+enum { K_PREP = 0, K_ATTN = 1, K_UPDATE = 2, K_APPLY = 3, K_TOK_PREP = 4, K_TOK_CHAIN = 5, K_TOK_READS = 6 };
 
 struct Timing {
     bool on = false;
@@ -100,6 +108,12 @@ cudaError_t timed(int kind, cudaStream_t st, F fn) {
 
 bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
+// Fault test (off by default): see hyb_attn_set_fault_test in the header.
+struct FaultTest {
+    int skip_v = 0;
+    unsigned long long wait_ns = 2000000000ull;
+} g_fault;
+
 // Opt each kernel into its dynamic shared memory once per device.
 template <typename K>
 cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
@@ -117,6 +131,9 @@ cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
     if (e == cudaSuccess) done[dev] = 1;
     return e;
 }
+
+// CTAs of the attention kernel along the query axis: two 128-query tiles each.
+unsigned attn_pairs(int T) { return (unsigned)(((T + tc::kTile - 1) / tc::kTile + 1) / 2); }
 
 template <int D, typename TIO>
 cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
@@ -215,23 +232,22 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
 }
 
 cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
-    using bf16 = __nv_bfloat16;
     static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
     constexpr int D = 128;
     cudaError_t e;
-    const size_t prep_smem = simt::PrepSmem<D, simt::prep_rows<true>()>::bytes;
-    if ((e = opt_in_smem(simt::prep_kernel<D, bf16, true>, prep_smem, done_prep)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return e;
     if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
     const uint64_t row_bytes = (uint64_t)a.H * D * 2;
     const uint64_t bh = (uint64_t)a.B * a.H;
-    CUtensorMap tq, tk, tv, tw, tphik, tout;
+    CUtensorMap tq, tk, tv, tw, tphik, tphiq, tout;
     if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
         (a.out && !map3d(&tout, a.out, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T)) ||
         !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
         !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
         !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
-        !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2))
+        !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2) ||
+        !map3d(&tphiq, a.phi_q, D, D, a.H, D * 2, D * D * 2))
         return cudaErrorInvalidValue;
     if (!a.out) tout = tq;  // not read: the attention kernel stores no bf16 output
     // Kernels of a pass are chained by programmatic dependent launch: prep waits
@@ -241,24 +257,24 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t pcfg = {};
-    pcfg.gridDim = dim3(D / simt::prep_rows<true>(), a.H, a.B);
-    pcfg.blockDim = dim3(simt::kThreads, 1, 1);
-    pcfg.dynamicSmemBytes = prep_smem;
+    pcfg.gridDim = dim3(1, a.H, a.B);
+    pcfg.blockDim = dim3(tc::prep::kThreads, 1, 1);
+    pcfg.dynamicSmemBytes = tc::prep::SMEM;
     pcfg.stream = st;
     pcfg.attrs = pdl;
     pcfg.numAttrs = 1;
     cudaError_t le = cudaSuccess;
-    e = timed(K_PREP, st, [&] { le = cudaLaunchKernelEx(&pcfg, simt::prep_kernel<D, bf16, true>, a, clean); });
+    e = timed(K_PREP, st, [&] { le = cudaLaunchKernelEx(&pcfg, tc::prep_tc_kernel, a, tphiq); });
     if (e != cudaSuccess) return e;
     if (le != cudaSuccess) return le;
     cudaLaunchConfig_t acfg = {};
-    acfg.gridDim = dim3((a.T + tc::kTile - 1) / tc::kTile, a.H, a.B);
-    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
-    acfg.dynamicSmemBytes = tc::attn::SMEM;
+    acfg.gridDim = dim3(attn_pairs(a.T), a.H, a.B);
+    acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::pp::SMEM;
     acfg.stream = st;
     acfg.attrs = pdl;
     acfg.numAttrs = 1;
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw, tout); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tw, tout); });
     if (e != cudaSuccess) return e;
     if (le != cudaSuccess) return le;
     if (clean) {
@@ -340,9 +356,86 @@ hyb_status pass_args(const hyb_attn_desc* desc, const void* q, const void* k, co
     a.partials = (float*)(ws + p.off_part);
     a.nsplit = p.nsplit;
     a.split_tokens = p.split_tokens;
+    a.wait_ns = g_fault.wait_ns;
+    a.dbg_skip_v = g_fault.skip_v;
     *args = a;
     *plan = p;
     return HYB_OK;
+}
+
+// ---- token-level access (clean passes) -------------------------------------------
+struct TokPlan {
+    size_t off_rec, off_out, total;
+    int nch;
+};
+
+TokPlan tok_plan(const hyb_attn_desc* d, const Plan& p) {
+    TokPlan t;
+    t.nch = (d->T + tok::kChunk - 1) / tok::kChunk;
+    const size_t rec_floats = p.D == 128 ? tok::Rec<128>::floats : tok::Rec<32>::floats;
+    const size_t recs = (size_t)d->B * d->H * t.nch * rec_floats * sizeof(float);
+    t.off_rec = align_up(p.total, 256);
+    t.off_out = align_up(t.off_rec + recs, 256);
+    t.total = align_up(t.off_out + (size_t)d->B * d->T * d->H * p.D * sizeof(float), 256);
+    return t;
+}
+
+template <int D, typename TIO>
+cudaError_t launch_token_level(LayerArgs a, const TokPlan& tp, char* ws, cudaStream_t st) {
+    static unsigned char done_prep[kMaxDevices], done_chain[kMaxDevices], done_reads[kMaxDevices];
+    cudaError_t e;
+    if ((e = opt_in_smem(tok::chunk_prep_kernel<D, TIO>, tok::PrepSmem<D>::bytes, done_prep)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tok::chunk_chain_kernel<D>, tok::ChainSmem<D>::bytes, done_chain)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tok::chunk_reads_kernel<D>, tok::ReadsSmem<D>::bytes, done_reads)) != cudaSuccess) return e;
+    float* rec = (float*)(ws + tp.off_rec);
+    float* oi = (float*)(ws + tp.off_out);
+    const dim3 cg(tp.nch, a.H, a.B);
+    e = timed(K_TOK_PREP, st, [&] {
+        tok::chunk_prep_kernel<D, TIO><<<cg, tok::kThreads, tok::PrepSmem<D>::bytes, st>>>(a, rec);
+    });
+    if (e != cudaSuccess) return e;
+    e = timed(K_TOK_CHAIN, st, [&] {
+        tok::chunk_chain_kernel<D><<<dim3(D / tok::kBand, a.H, a.B), D, tok::ChainSmem<D>::bytes, st>>>(a, rec);
+    });
+    if (e != cudaSuccess) return e;
+    e = timed(K_TOK_READS, st, [&] {
+        tok::chunk_reads_kernel<D><<<cg, tok::kThreads, tok::ReadsSmem<D>::bytes, st>>>(a, rec, oi);
+    });
+    if (e != cudaSuccess) return e;
+    // the attention kernel adds the token-level read instead of Q W
+    a.inter = 0;
+    a.oi_ext = oi;
+    if constexpr (D == 128) {
+        static unsigned char done_attn[kMaxDevices];
+        if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return e;
+        const uint64_t row_bytes = (uint64_t)a.H * D * 2;
+        CUtensorMap tq, tk, tv, tout;
+        if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            (a.out && !map3d(&tout, a.out, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T)))
+            return cudaErrorInvalidValue;
+        if (!a.out) tout = tq;
+        cudaLaunchConfig_t acfg = {};
+        acfg.gridDim = dim3(attn_pairs(a.T), a.H, a.B);
+        acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
+        acfg.dynamicSmemBytes = tc::pp::SMEM;
+        acfg.stream = st;
+        cudaError_t le = cudaSuccess;
+        // tq stands in for the unused W map
+        e = timed(K_ATTN, st,
+                  [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tq, tout); });
+        if (e != cudaSuccess) return e;
+        if (le != cudaSuccess) return le;
+    } else {
+        static unsigned char done_attn[kMaxDevices];
+        const size_t attn_smem = simt::AttnSmem<D>::bytes;
+        if ((e = opt_in_smem(simt::attn_kernel<D, TIO>, attn_smem, done_attn)) != cudaSuccess) return e;
+        const dim3 agrid((a.T + simt::AttnSmem<D>::BQ - 1) / simt::AttnSmem<D>::BQ, a.H, a.B);
+        e = timed(K_ATTN, st, [&] { simt::attn_kernel<D, TIO><<<agrid, simt::kThreads, attn_smem, st>>>(a); });
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
 }
 
 hyb_status launch_pass(const LayerArgs& a, const Plan& p, int clean_pass, void* stream) {
@@ -418,10 +511,12 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.v = v_cache;
     a.out = out;
     a.flags = (unsigned*)workspace;
+    a.wait_ns = g_fault.wait_ns;
+    a.dbg_skip_v = g_fault.skip_v;
 
     static unsigned char done_attn[kMaxDevices];
     cudaError_t e;
-    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
+    if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
     const uint64_t row_bytes = (uint64_t)H * D * 2;
     CUtensorMap tq, tk, tv, tout;
     if (!map3d(&tq, q, (uint64_t)H * D, T, B, row_bytes, row_bytes * T) ||
@@ -430,13 +525,13 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
         !map3d(&tout, out, (uint64_t)H * D, T, B, row_bytes, row_bytes * T))
         return HYB_ERR_CUDA;
     cudaLaunchConfig_t acfg = {};
-    acfg.gridDim = dim3((T + tc::kTile - 1) / tc::kTile, H, B);
-    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
-    acfg.dynamicSmemBytes = tc::attn::SMEM;
+    acfg.gridDim = dim3(attn_pairs(T), H, B);
+    acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::pp::SMEM;
     acfg.stream = st;
     cudaError_t le = cudaSuccess;
     // tq stands in for the unused W map
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tq, tout); });
     if (e != cudaSuccess || le != cudaSuccess) return HYB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
@@ -488,6 +583,38 @@ hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc, const void* q, cons
                         nullptr, nullptr, workspace, workspace_bytes, stream, mix);
 }
 
+size_t hyb_attn_token_level_workspace_bytes(const hyb_attn_desc* desc) {
+    Plan p;
+    if (make_plan(desc, &p) != HYB_OK) return 0;
+    return tok_plan(desc, p).total;
+}
+
+hyb_status hyb_attn_forward_token_level(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                                        const void* phi_q, const void* phi_k, const void* phi_v,
+                                        const float* gate_logits, const float* beta_logits, float* state,
+                                        int clean_pass, void* out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    if (!out) return HYB_ERR_INVALID;
+    Plan p;
+    hyb_status s = make_plan(desc, &p);
+    if (s != HYB_OK) return s;
+    const TokPlan tp = tok_plan(desc, p);
+    if (workspace && workspace_bytes < tp.total) return HYB_ERR_WORKSPACE;
+    LayerArgs a;
+    s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out, nullptr,
+                  nullptr, workspace, workspace_bytes, nullptr, &a, &p);
+    if (s != HYB_OK) return s;
+    // a query-only pass reads the frame-start state with every token: it is the
+    // frame-level pass
+    if (!clean_pass) return launch_pass(a, p, 0, stream);
+    cudaError_t e;
+    if (p.bf16)
+        e = launch_token_level<128, __nv_bfloat16>(a, tp, (char*)workspace, (cudaStream_t)stream);
+    else
+        e = launch_token_level<32, float>(a, tp, (char*)workspace, (cudaStream_t)stream);
+    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
 hyb_status hyb_attn_get_device_status(const void* workspace, void* stream) {
     if (!workspace) return HYB_ERR_INVALID;
     if (!aligned16(workspace)) return HYB_ERR_ALIGN;
@@ -500,6 +627,14 @@ hyb_status hyb_attn_get_device_status(const void* workspace, void* stream) {
     if (flags & FLAG_INTERNAL) return HYB_ERR_CUDA;
     if (flags & FLAG_TIMEOUT) return HYB_ERR_TIMEOUT;
     if (flags & FLAG_NONFINITE) return HYB_WARN_NONFINITE;
+    return HYB_OK;
+}
+
+hyb_status hyb_attn_set_fault_test(int skip_v_loads, unsigned wait_limit_us) {
+    if (skip_v_loads != 0 && skip_v_loads != 1) return HYB_ERR_INVALID;
+    if (wait_limit_us > 10u * 1000u * 1000u) return HYB_ERR_INVALID;
+    g_fault.skip_v = skip_v_loads;
+    g_fault.wait_ns = wait_limit_us ? (unsigned long long)wait_limit_us * 1000ull : 2000000000ull;
     return HYB_OK;
 }
 
@@ -558,7 +693,8 @@ hyb_status hyb_attn_timing_end(hyb_attn_timing* out) {
 
 const char* hyb_attn_kernel_name(int kernel) {
     static const char* names[HYB_NUM_KERNELS] = {"prep", "intra_frame_attention", "delta_update",
-                                                 "delta_update_apply"};
+                                                 "delta_update_apply", "token_chunk_prep", "token_chain",
+                                                 "token_reads"};
     return (kernel >= 0 && kernel < HYB_NUM_KERNELS) ? names[kernel] : nullptr;
 }
 

@@ -26,15 +26,13 @@ namespace simt {
 constexpr int kThreads = 256;
 
 // ---------------------------------------------------------------- prep
-// grid (D/R, H, B): block x computes rows k0..k0+R-1 of W = phi_q^T S (row-major;
-// fp32 for the SIMT path, a bf16 hi + lo pair for the tensor path).  S and the
-// block's R columns of phi_q are staged in shared memory; each warp owns R/8
-// rows of W and every lane D/32 consecutive columns.  The tensor path takes
-// R = 64 (two blocks per head), so that the attention kernel launched behind it
-// finds most SMs free; the SIMT path takes R = 16.
+// grid (D/R, H, B): block x computes rows k0..k0+R-1 of W = phi_q^T S (row-major
+// fp32).  S and the block's R columns of phi_q are staged in shared memory; each
+// warp owns R/8 rows of W and every lane D/32 consecutive columns.  (The
+// tensor-core path computes W with tcgen05 in tc_kernels.cuh.)
 constexpr int kRows = 16;
 template <bool kSplitOut>
-__host__ __device__ constexpr int prep_rows() { return kSplitOut ? 64 : 16; }
+__host__ __device__ constexpr int prep_rows() { return 16; }
 
 template <int D, int R>
 struct PrepSmem {
@@ -43,6 +41,7 @@ struct PrepSmem {
 
 template <int D, typename TIO, bool kSplitOut>
 __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) {
+    static_assert(!kSplitOut, "the bf16 hi + lo W is written by the tensor-core prep kernel");
     constexpr int NC = D / 32;
     constexpr int R = prep_rows<kSplitOut>();
     constexpr int RW = R / (kThreads / 32);  // rows of W per warp
@@ -53,12 +52,6 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
     const int b = blockIdx.z, h = blockIdx.y, k0 = blockIdx.x * R;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
-    if constexpr (kSplitOut) {
-        // tensor path, launched as a programmatic dependent: wait until the
-        // previous kernel (which may write the state) has completed before
-        // reading S_{N-1}
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-    }
     // all loads of a thread are issued before any shared-memory store: the
     // stores go through generic pointers, which would otherwise serialise them
     {
@@ -81,13 +74,6 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
         for (int u = 0; u < NP; ++u) Ph[tid + u * kThreads] = pv[u];
     }
     __syncthreads();
-    if constexpr (kSplitOut) {
-        // S_{N-1} is in shared memory: only now may the attention kernel start,
-        // and through it the delta update that overwrites the state in place
-        // (it is launched once every attention CTA has started).  The attention
-        // kernel reads W only after this grid has completed.
-        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    }
     // each warp owns rows r0..r0+RW-1 of W; each lane NC consecutive columns
     const int r0 = RW * warp;
     float acc[RW][NC];
@@ -131,25 +117,10 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(LayerArgs a, int clean) 
 #pragma unroll
     for (int rr = 0; rr < RW; ++rr) {
         const size_t row = bh * D * D + (size_t)(k0 + r0 + rr) * D + NC * lane;
-        if constexpr (kSplitOut) {
-            // row-major W as a bf16 hi + lo pair
-            uint32_t hi[NC / 2], lo[NC / 2];
 #pragma unroll
-            for (int c = 0; c < NC / 2; ++c) {
-                const __nv_bfloat162 hv = __floats2bfloat162_rn(acc[rr][2 * c], acc[rr][2 * c + 1]);
-                const __nv_bfloat162 lv = __floats2bfloat162_rn(acc[rr][2 * c] - __low2float(hv),
-                                                                acc[rr][2 * c + 1] - __high2float(hv));
-                hi[c] = *reinterpret_cast<const uint32_t*>(&hv);
-                lo[c] = *reinterpret_cast<const uint32_t*>(&lv);
-            }
-            *reinterpret_cast<uint2*>(a.WT_hi + row) = make_uint2(hi[0], hi[1]);
-            *reinterpret_cast<uint2*>(a.WT_lo + row) = make_uint2(lo[0], lo[1]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < NC; ++c) a.W[row + c] = acc[rr][c];
-        }
+        for (int c = 0; c < NC; ++c) a.W[row + c] = acc[rr][c];
     }
-    if (clean && !kSplitOut) {
+    if (clean) {
         // the fp32 update reads S_{N-1} from this copy (it writes the state in place)
         float4* dst = reinterpret_cast<float4*>(a.S_prev + bh * D * D + (size_t)k0 * D);
         for (int i = tid; i < R * D / 4; i += kThreads)
@@ -244,15 +215,27 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(LayerArgs a) {
     for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < NC; ++c) oe[r][c] = 0.f;
-    for (int kk = 0; kk < D; ++kk) {
-        float w[NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) w[c] = W[kk * D + lane + 32 * c];
+    if (a.oi_ext) {
+        // token-level access: the read was computed by the token-level kernels
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-            const float qv = qrow[r * D + kk];
+            const int t = q0 + warp * 8 + r;
+            if (t >= T) continue;
+            const float* src = a.oi_ext + (((size_t)b * T + t) * a.H + h) * D;
 #pragma unroll
-            for (int c = 0; c < NC; ++c) oe[r][c] = fmaf(qv, w[c], oe[r][c]);
+            for (int c = 0; c < NC; ++c) oe[r][c] = src[lane + 32 * c];
+        }
+    } else {
+        for (int kk = 0; kk < D; ++kk) {
+            float w[NC];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) w[c] = W[kk * D + lane + 32 * c];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const float qv = qrow[r * D + kk];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) oe[r][c] = fmaf(qv, w[c], oe[r][c]);
+            }
         }
     }
 #pragma unroll

@@ -47,13 +47,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Every wait is bounded.  A wait that does not complete within kWaitNs sets the
+// Every wait is bounded.  A wait that does not complete within limit_ns (kWaitNs
+// unless the caller passes its own) sets the
 // block's abort word and the workspace's TIMEOUT flag and returns false; once
 // abort is set, every other wait of the block returns false promptly.
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_word,
-                                          unsigned* gflags) {
+                                          unsigned* gflags, uint64_t limit_ns = kWaitNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -61,7 +62,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (mbar_try_wait(a, parity)) return true;
         if ((it & 63) == 0) {
             if (*abort_word) return false;
-            if (globaltimer_ns() - t0 > kWaitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort_word = 1;
                 atomicOr(gflags, FLAG_TIMEOUT);
                 return false;

@@ -1,37 +1,13 @@
-// tc_kernels.cuh -- tensor-core (tcgen05 / TMEM / TMA) kernels of the hybrid
-// layer for bf16 I/O and d = 128 on sm_100a.
+// tc_kernels.cuh -- tensor-core (tcgen05 / TMEM / TMA) delta update of the
+// hybrid layer for bf16 I/O and d = 128 on sm_100a.
 //
 // Source: "Technical summary: Attend Locally, Remember Linearly (ARL2)",
 // gist.science/ar/paper/2605.16579, §2.1 (intra-frame softmax branch,
 // inter-frame read O_inter = Q' S_{N-1}, gated delta update) and §2.2
 // (frame-level access: all tokens read the pre-update state).
 //
-// intra_frame_attention: one CTA per (128-query tile, head, batch), 11 warps.
-// Warp 8 streams Q and the K ring, warp 10 the V ring, with TMA into
-// 128B-swizzled shared memory; warp 9 issues the tcgen05 MMAs; warps 0-7 run
-// the online softmax, a query row per pair of threads (warps w and w+4, 64
-// scores each in registers).  Near the end of the key loop the Q tile is
-// multiplied by W = phi_q^T S_{N-1} (a two-term bf16 split W_hi + W_lo, row
-// major: an MN-major B operand), so the inter-frame read lands in TMEM next to
-// the softmax accumulator and the epilogue writes out = O_intra + O_inter once.
-//   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
-//                 [384,448) Q, [448,512) P (bf16, two per 32-bit column: the
-//                 A operands of S = Q K^T and O += P V).  Q is copied from
-//                 shared memory into TMEM once; as soon as the softmax has S_j
-//                 in registers the MMA warp issues S_{j+2} into its buffer, so
-//                 scores run a tile ahead of the softmax, and the softmax loads
-//                 S_{j+1} while it hands P_j over.
-//   Softmax: exponents against a running offset (the first tile's row max),
-//                 moved only when a tile's partial sum over a half row leaves
-//                 [0, 2^63); all exponentials on the MUFU pipe.
-//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Near the end W_hi
-//                 and W_lo take the K stages of key tiles n-3 and n-2 (unused
-//                 stages when n < 3) and O_inter = Q W_hi + Q W_lo goes to the
-//                 S buffer the last tile does not use while the softmax works
-//                 on the last two tiles; the bf16 output tile is assembled in
-//                 the Q buffer and written with two TMA stores.
-//   Every CTA signals at entry that the next kernel (the delta update, which
-//   reads none of this kernel's outputs) may start on idle SMs.
+// The attention kernel is in tc_attention.cuh; this file holds the operand
+// descriptors both use and the delta update.
 //
 // delta_update: one cluster per (head, batch), one CTA per token split.  Per
 // 128-token tile: K~ = K phi_k^T on the tensor core, row L2-normalisation and
@@ -55,24 +31,6 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr uint32_t kHalf = kTileBytes / 2;      // one 128 x 64 TMA box
 constexpr int kMaxClusterRanks = 8;             // token splits per (b, h) in the update
 
-// ============================================================== attention
-namespace attn {
-constexpr int kKStages = 3;                    // K ring depth
-constexpr int kVStages = 3;                    // V ring depth
-constexpr uint32_t Q = 0;
-constexpr uint32_t K0 = Q + kTileBytes;
-constexpr uint32_t V0 = K0 + kKStages * kTileBytes;
-constexpr uint32_t BAR = V0 + kVStages * kTileBytes;
-constexpr uint32_t XCH = BAR + 256;            // softmax pair exchange: [2 parity][2 halves][128 rows] floats
-constexpr uint32_t XFL = XCH + 2048;           // and codes [2][2][128] bytes
-constexpr uint32_t SMEM = XFL + 512;           // 232,192 B
-constexpr int kSoftmaxThreads = 256;           // warps 0-7: rows 32(w&3)..+31, column half w>>2
-constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadVWarp = 10;
-constexpr int kThreads = 352;
-enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12, B_SFULL = 15,
-       B_SREAD = 17, B_QTM = 19, B_PFULL = 20, B_PVDONE = 21, B_COUNT = 22 };
-static_assert(B_COUNT * 8 + 8 <= 256, "barrier block");
-}  // namespace attn
 
 // K-major operand, 128 rows x 128 bf16 stored as two 64-column swizzled boxes:
 // descriptor of the 16-column slice kk (0..7).
@@ -93,415 +51,6 @@ __device__ __forceinline__ float row_max(const float* x) {
 #pragma unroll
     for (int c = 8; c < N; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
     return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-}
-
-// p = 2^(x * scale + neg_m) for N scores, as N/2 bf16 pairs (round to
-// nearest) in pk; returns the sum of p in fp32 (the exponentials on the MUFU
-// pipe, the pair conversion one instruction per two values).
-template <int N>
-__device__ __forceinline__ float exp_scores(const float* x, float scale, float neg_m, uint32_t* pk) {
-    float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < N / 2; ++k) {
-        const float e0 = ex2(fmaf(x[2 * k], scale, neg_m));
-        const float e1 = ex2(fmaf(x[2 * k + 1], scale, neg_m));
-        l4[(2 * k) & 3] += e0;
-        l4[(2 * k + 1) & 3] += e1;
-        pk[k] = pack_bf16(e0, e1);
-    }
-    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
-}
-
-__global__ void __launch_bounds__(attn::kThreads, 1)
-    attention_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
-    using namespace attn;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    // 128B-swizzled tiles need a 1024-byte aligned base (the dynamic window starts
-    // after the 1 KB reserved block); report and leave if it is not
-    if (smem_u32(smem) & 1023u) {
-        if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
-        return;
-    }
-    // the delta update of this pass does not read anything this kernel writes:
-    // it may start on SMs this grid leaves idle
-    pdl_launch_dependents();
-    const uint32_t sb = smem_u32(smem);
-    uint64_t* bars = (uint64_t*)(smem + BAR);
-    uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
-    volatile int* abort_word = (volatile int*)(tmem_slot + 1);
-    volatile int* epi_bad = (volatile int*)(tmem_slot + 2);  // a softmax warp missed its epilogue
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int T = a.T;
-    const int q0 = qt_ * kTile;
-    const int n = (a.T_kv + kTile - 1) / kTile;  // key tiles
-    const bool inter = a.inter != 0;             // add O_inter = Q W (hybrid layer)
-    const int bh = b * a.H + h;
-    // K stages that receive W_hi / W_lo at the end (free once the scores of key
-    // tiles n-3 / n-2 are computed; stages no tile uses when n is small)
-    const int wst_hi = n >= 3 ? (n - 3) % kKStages : 2;
-    const int wst_lo = n >= 2 ? (n - 2) % kKStages : 1;
-
-    if (threadIdx.x == kLoadWarp * 32) {
-        // the producer initialises the barriers and starts the first loads
-        // before the block synchronises (the loads land on its own barriers)
-        for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(&bars[i],
-                      (i == B_PFULL || i == B_QTM || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads : 1);
-        *abort_word = 0;
-        *epi_bad = 0;
-        fence_mbar_init();
-        fence_async_smem();
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        const int xh = h * 128;
-        mbar_expect_tx(&bars[B_Q], kTileBytes);
-        tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0, b);
-        tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
-        for (int j = 0; j < kKStages && j < n; ++j) {
-            mbar_expect_tx(&bars[B_KFULL + j], kTileBytes);
-            tma_load_3d(sb + K0 + j * kTileBytes, &tm_k, &bars[B_KFULL + j], xh, j * kTile, b);
-            tma_load_3d(sb + K0 + j * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + j], xh + 64, j * kTile, b);
-        }
-    }
-    if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    // S buffers 0 / 1, O, Q and P as bf16 pairs (the A operands of the score
-    // and value products)
-    const uint32_t tS0 = tmem, tO = tmem + 256, tQ = tmem + 384, tP = tmem + 448;
-    const uint32_t tOI = tS0 + (n & 1) * 128;  // the S buffer the last tile does not use
-
-    if (warp == kLoadVWarp) {
-        // ------------------------------------------------ TMA producer: V ring
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_v);
-            const int xh = h * 128;
-            for (int j = 0; j < n; ++j) {
-                const int vs = j % kVStages;
-                if (j >= kVStages &&
-                    !mbar_wait(&bars[B_VEMPTY + vs], ((j / kVStages) + 1) & 1, abort_word, a.flags))
-                    break;
-                mbar_expect_tx(&bars[B_VFULL + vs], kTileBytes);
-                tma_load_3d(sb + V0 + vs * kTileBytes, &tm_v, &bars[B_VFULL + vs], xh, j * kTile, b);
-                tma_load_3d(sb + V0 + vs * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + vs], xh + 64, j * kTile, b);
-            }
-        }
-        __syncwarp();
-    } else if (warp == kLoadWarp) {
-        // ------------------------------------------------ TMA producer: Q, K ring, W
-        // (its own warp, so K tiles run ahead of the V ring's waits)
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_w);
-            const int xh = h * 128;
-            bool ok = true;
-            for (int j = kKStages; j < n && ok; ++j) {  // Q and K_0..K_2 were issued at entry
-                const int ks = j % kKStages;
-                if (!(ok = mbar_wait(&bars[B_KEMPTY + ks], ((j / kKStages) + 1) & 1, abort_word, a.flags))) break;
-                mbar_expect_tx(&bars[B_KFULL + ks], kTileBytes);
-                tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, j * kTile, b);
-                tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64, j * kTile, b);
-            }
-            // W_hi / W_lo (row-major, MN-major operands) into K stages freed by S_{n-3} / S_{n-2}
-            const int nbh = a.B * a.H;
-            if (inter && ok && n >= 3)
-                ok = mbar_wait(&bars[B_KEMPTY + wst_hi], ((n - 3) / kKStages) & 1, abort_word, a.flags);
-            if (inter && ok && n >= 2)
-                ok = mbar_wait(&bars[B_KEMPTY + wst_lo], ((n - 2) / kKStages) & 1, abort_word, a.flags);
-            // W comes from the prep kernel, which may still be running when this
-            // grid starts (programmatic dependent launch): wait for it here
-            if (inter) pdl_wait_primary();
-            if (inter && ok) {
-                mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
-                tma_load_3d(sb + K0 + wst_hi * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
-                tma_load_3d(sb + K0 + wst_hi * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
-                tma_load_3d(sb + K0 + wst_lo * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
-                tma_load_3d(sb + K0 + wst_lo * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
-            }
-        }
-        __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------ MMA issuer
-        // S_j = Q K_j^T into S buffer j&1 (A = Q from TMEM); S_{j+2} reuses the
-        // buffer as soon as the softmax has S_j in registers, so scores run a
-        // tile ahead.  O += P_j V_j once P_j is in TMEM.
-        if (lane == 0) {
-            constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            // S_0 and S_1 take Q from shared memory (no wait for its copy into TMEM)
-            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags);
-            bool q_in_tmem = false;
-            for (int j = 0; j < 2 && j < n && ok; ++j) {
-                if (!(ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK,
-                             kk > 0);
-                mma_commit(&bars[B_SFULL + j]);
-                mma_commit(&bars[B_KEMPTY + j]);
-            }
-            for (int j = 0; j < n && ok; ++j) {
-                const int sbuf = j & 1;
-                if (j + 2 < n) {
-                    const int ks = (j + 2) % kKStages;
-                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags))) break;
-                    if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags))) break;
-                    if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tS0 + sbuf * 128, tQ + kk * 8, kmajor_desc(sb + K0 + ks * kTileBytes, kk), ID_KK,
-                                    kk > 0);
-                    mma_commit(&bars[B_SFULL + sbuf]);
-                    mma_commit(&bars[B_KEMPTY + ks]);
-                }
-                if (inter && j == (n >= 2 ? n - 2 : 0)) {
-                    // O_inter = Q W_hi + Q W_lo into S buffer n&1 (free once the
-                    // softmax has S_{n-2} in registers; unused when n == 1), run
-                    // while the softmax works on the last two tiles
-                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags))) break;
-                    if (n >= 2 &&
-                        !(ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags)))
-                        break;
-                    if (!(ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
-                    mma_commit(&bars[B_OIDONE]);
-                }
-                const int vs = j % kVStages;
-                if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags))) break;
-                if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tO, tP + kk * 8, mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
-                mma_commit(&bars[B_PVDONE]);
-                mma_commit(&bars[B_VEMPTY + vs]);
-            }
-            // drain: every MMA issued so far completes before TMEM is released
-            mma_commit(&bars[B_Q]);
-            uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(smem_u32(&bars[B_Q]), 1) && globaltimer_ns() - t0 < kWaitNs) {
-            }
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------ softmax + epilogue
-        // Warps w and w+4 share query rows 32(w&3)..+31 (TMEM lanes); warp w>>2
-        // takes score and output columns 64(w>>2)..+63, so two softmax warps
-        // per SM sub-partition interleave their exponentials.  S_j is released
-        // (SREAD) as soon as it is in registers, so S_{j+2} is computed while
-        // this tile is exponentiated, and S_{j+1} is loaded before P_j is
-        // handed to the MMA warp.
-        //
-        // Offset: exponents are taken against a running offset m (log2 units)
-        // that is the row max of the first tile and moves only when a tile's
-        // partial sum over a half leaves [0, 2^63): the tile is then redone
-        // against the row's max and O, l are rescaled.  Every value stays
-        // finite, P <= 2^63, and the result is the same softmax (the offset
-        // cancels in O / l).
-        //
-        // The two warps of a pair exchange a code per row and tile (0: a wait
-        // failed, 1: ok, 2: offset too low) at their pair barrier and take the
-        // same path from it; a warp whose wait failed keeps arriving at the
-        // pair barriers to the end, so neither warp ever waits for the other
-        // without a partner.
-        const int g = warp & 3, hf = warp >> 2;
-        const int r = g * 32 + lane;
-        const int pair_bar = 1 + g;
-        const uint32_t lrow = (uint32_t)(g * 32) << 16;
-        const uint32_t cs = hf * 64;
-        float* xch = (float*)(smem + XCH);
-        uint8_t* xfl = smem + XFL;
-        const int mine = hf * 128 + r, theirs = (hf ^ 1) * 128 + r;  // + parity * 256
-        const float scale = a.sm_scale_log2;
-        float m = 0.f, l = 0.f;
-        float x[64];
-        // this half of Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags));
-        if (ok) {
-            uint32_t qv[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hf * kHalf + sw128_offset(r, c));
-                qv[4 * c] = v.x;
-                qv[4 * c + 1] = v.y;
-                qv[4 * c + 2] = v.z;
-                qv[4 * c + 3] = v.w;
-            }
-            tmem_st32u(tQ + lrow + hf * 32, qv);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[B_QTM]);
-        }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags));
-        if (ok) {
-            tc_fence_after();
-            tmem_ld32(tS0 + lrow + cs, x);
-            tmem_ld32(tS0 + lrow + cs + 32, x + 32);
-        }
-        for (int j = 0; j < n; ++j) {
-            const int s = j & 1;
-            const bool w_ok = ok;
-            uint32_t pk[32];
-            float lt = 0.f;
-            if (w_ok) {
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
-                const int valid = a.T_kv - j * kTile - (int)cs;
-                if (valid < 64) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (c >= valid) x[c] = -INFINITY;
-                }
-            }
-            if (j == 0) {
-                // the first tile's row max over both halves sets the offset
-                const float hm = w_ok ? row_max<64>(x) : -INFINITY;
-                xch[mine] = hm;
-                named_bar_sync(pair_bar, 64);
-                m = fmaxf(hm, xch[theirs]) * scale;
-            }
-            bool redo_h = false;
-            if (w_ok) {
-                lt = exp_scores<64>(x, scale, -m, pk);
-                redo_h = !(lt < 9.2233720e18f);  // >= 2^63, inf or NaN
-            }
-            xfl[s * 256 + mine] = w_ok ? (redo_h ? 2 : 1) : 0;
-            named_bar_sync(pair_bar, 64);
-            const uint8_t pc = xfl[s * 256 + theirs];
-            ok = __all_sync(0xffffffffu, w_ok && pc != 0);  // the same in both warps of the pair
-            const bool redo = ok && (redo_h || pc == 2);
-            const bool any_redo = __any_sync(0xffffffffu, redo);
-            float f = 1.0f;
-            if (any_redo) {
-                // the offset is too low for this tile (or a score is not finite):
-                // move it to the row's max and redo P_j; O is rescaled below
-                const float hm = redo ? row_max<64>(x) * scale : -INFINITY;
-                xch[s * 256 + mine] = hm;
-                named_bar_sync(pair_bar, 64);
-                if (redo) {
-                    const float mn = fmaxf(m, fmaxf(hm, xch[s * 256 + theirs]));
-                    f = ex2(m - mn);
-                    m = mn;
-                }
-                lt = exp_scores<64>(x, scale, -m, pk);
-            }
-            if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
-            l = fmaf(l, f, lt);
-            // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE], (j - 1) & 1, abort_word, a.flags));
-                if (!ok) continue;
-                tc_fence_after();
-            }
-            if (any_redo && j > 0) {
-#pragma unroll 1
-                for (int c = 0; c < 64; c += 32) {
-                    float o[32];
-                    tmem_ld32(tO + lrow + cs + c, o);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) o[q] *= f;
-                    tmem_st32(tO + lrow + cs + c, o);
-                }
-            }
-            tmem_st32u(tP + lrow + hf * 32, pk);
-            // this half of S_{j+1} into registers while P_j is being stored
-            if (j + 1 < n) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + (s ^ 1)], ((j + 1) >> 1) & 1, abort_word,
-                                                       a.flags));
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t src = tS0 + (s ^ 1) * 128 + lrow + cs;
-                    tmem_ld32(src, x);
-                    tmem_ld32(src + 32, x + 32);
-                }
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            if (ok) mbar_arrive(&bars[B_PFULL]);
-        }
-        // epilogue: out = O / l + O_inter for this half of the row
-        if (ok) tmem_ld_wait();
-        bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags);
-        e_ok = __all_sync(0xffffffffu, e_ok && (!inter || mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags)));
-        // row sum over the two halves (slot parity n&1: its last readers passed
-        // the pair barrier of tile n-1)
-        xch[(n & 1) * 256 + mine] = l;
-        xfl[(n & 1) * 256 + mine] = e_ok ? 1 : 0;
-        named_bar_sync(pair_bar, 64);
-        const bool both = __all_sync(0xffffffffu, e_ok && xfl[(n & 1) * 256 + theirs] != 0);
-        if (both) {
-            tc_fence_after();
-            const float inv_l = 1.0f / (l + xch[(n & 1) * 256 + theirs]);  // commutative: the same in both halves
-            // out = a O_intra + O_inter (the inter gain c is folded into W); a = 1 without a mix
-            const float inv_out = a.mix ? inv_l * a.mix[bh * 2] : inv_l;
-            const int t = q0 + r;
-            const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + cs;
-            float o[64], e[64];
-            tmem_ld32(tO + lrow + cs, o);
-            tmem_ld32(tO + lrow + cs + 32, o + 32);
-            if (inter) {
-                tmem_ld32(tOI + lrow + cs, e);
-                tmem_ld32(tOI + lrow + cs + 32, e + 32);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 64; ++q) e[q] = 0.f;
-            }
-            tmem_ld_wait();
-            if (a.out) {
-                // bf16 half-row into box hf of the (free) Q buffer, 128B-swizzled
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16(o[8 * q + 0] * inv_out + e[8 * q + 0], o[8 * q + 1] * inv_out + e[8 * q + 1]);
-                    w.y = pack_bf16(o[8 * q + 2] * inv_out + e[8 * q + 2], o[8 * q + 3] * inv_out + e[8 * q + 3]);
-                    w.z = pack_bf16(o[8 * q + 4] * inv_out + e[8 * q + 4], o[8 * q + 5] * inv_out + e[8 * q + 5]);
-                    w.w = pack_bf16(o[8 * q + 6] * inv_out + e[8 * q + 6], o[8 * q + 7] * inv_out + e[8 * q + 7]);
-                    *reinterpret_cast<uint4*>(smem + Q + hf * kHalf + sw128_offset(r, q)) = w;
-                }
-                fence_async_smem();
-            }
-            if (a.out_intra && t < T) {
-                float4* di = reinterpret_cast<float4*>(a.out_intra + row);
-                float4* de = reinterpret_cast<float4*>(a.out_inter + row);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
-                                        o[4 * q + 3] * inv_l);
-                    de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
-                }
-            }
-        }
-        // every softmax warp reaches this barrier (no early exit); the tile is
-        // stored only if all eight wrote their half-rows
-        if (!both && lane == 0) *epi_bad = 1;
-        named_bar_sync(5, kSoftmaxThreads);
-        if (a.out && threadIdx.x == 0 && *epi_bad == 0) {
-            // rows past T are clipped by the tensor map
-            tma_store_3d(&tm_o, sb + Q, h * 128, q0, b);
-            tma_store_3d(&tm_o, sb + Q + kHalf, h * 128 + 64, q0, b);
-            bulk_commit_group();
-            bulk_wait_read_all();
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ============================================================== delta update
@@ -539,7 +88,8 @@ constexpr uint32_t SMEM = XSS + 2048 + 512;               // 232,192 B
 constexpr int kNormThreads = 256;                         // warps 0-7
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
-enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_OPSFULL, B_OPSFREE, B_PARK, B_DELTA, B_COUNT };
+enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_KTFULL1, B_KTREAD, B_KTREAD1, B_OPSFULL, B_OPSFREE,
+       B_PARK, B_DELTA, B_COUNT };
 static_assert(RED + 128 * 128 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
 // byte offset of float4 chunk q (0..31) of row `row` in RED
 __device__ __forceinline__ uint32_t red_off(int row, int q) {
@@ -604,7 +154,8 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     for (int u = 0; u < 8; ++u) g0[u] = (threadIdx.x + u * kThreads < T) ? gl[threadIdx.x + u * kThreads] : 0.f;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_OPSFULL ? kNormThreads : 1);
+        for (int i = 0; i < B_COUNT; ++i)
+            mbar_init(&bars[i], (i == B_OPSFULL || i == B_KTREAD || i == B_KTREAD1) ? kNormThreads : 1);
         *abort_word = 0;
         fence_mbar_init();
     }
@@ -613,7 +164,10 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tKT = tmem, tG = tmem + 128, tP = tmem + 256;
+    // K~ of tile i in buffer i & 1 (columns [0,128) or [384,512)), so the K phi_k^T
+    // product of the next tile runs while this one is normalised
+    const uint32_t tG = tmem + 128, tP = tmem + 256;
+    auto tKT = [&](int i) { return (i & 1) ? tmem + 384 : tmem; };
 
     uint4 pv[8];  // phi_v staging (normalisation warps)
     // ------------------------------------------------------------ tile loop
@@ -643,25 +197,48 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         if (lane == 0 && nt > 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_MNMN = idesc_bf16(128, 128, 1, 1);
-            bool ok = mbar_wait(&bars[B_PHI], 0, abort_word, a.flags);
-            for (int i = 0; i < nt && ok; ++i) {
-                const uint32_t par = i & 1;
-                if (!mbar_wait(&bars[B_KFULL], par, abort_word, a.flags)) break;
+            // K~(i+1) = K_{i+1} phi_k^T is issued ahead of tile i's G and P products,
+            // so the next tile's normalisation can start while they run
+            bool ok = mbar_wait(&bars[B_PHI], 0, abort_word, a.flags) &&
+                      mbar_wait(&bars[B_KFULL], 0, abort_word, a.flags);
+            if (ok) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tKT, kmajor_desc(sb + KT, kk), kmajor_desc(sb + PHI, kk), ID_KK, kk > 0);
+                    mma_bf16(tKT(0), kmajor_desc(sb + KT, kk), kmajor_desc(sb + PHI, kk), ID_KK, kk > 0);
                 mma_commit(&bars[B_KTFULL]);
                 mma_commit(&bars[B_KFREE]);
-                if (!mbar_wait(&bars[B_OPSFULL], par, abort_word, a.flags)) break;
-                if (!mbar_wait(&bars[B_VFULL], par, abort_word, a.flags)) break;
+            }
+            for (int i = 0; i < nt && ok; ++i) {
+                if (i + 1 < nt) {
+                    if (!(ok = mbar_wait(&bars[B_KFULL], (i + 1) & 1, abort_word, a.flags))) break;
+                    // the buffer of K~(i+1) was last read by the normalisation of tile i-1
+                    if (i >= 1 && !(ok = mbar_wait(&bars[B_KTREAD + ((i + 1) & 1)], ((i - 1) >> 1) & 1,
+                                                   abort_word, a.flags)))
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tKT(i + 1), kmajor_desc(sb + KT, kk), kmajor_desc(sb + PHI, kk), ID_KK, kk > 0);
+                    mma_commit(&bars[B_KTFULL + ((i + 1) & 1)]);
+                    mma_commit(&bars[B_KFREE]);
+                }
+                if (!(ok = mbar_wait(&bars[B_OPSFULL], i & 1, abort_word, a.flags))) break;
                 tc_fence_after();
+                // G first: it does not need this tile's V, whose load starts only
+                // once the previous tile's P products have read the V buffer
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t acc = (i > 0 || kk > 0);
                     mma_bf16(tG, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + KH, kk), ID_MNMN, acc);
                     mma_bf16(tG, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + KL, kk), ID_MNMN, 1);
                     mma_bf16(tG, mnmajor_desc(sb + AL, kk), mnmajor_desc(sb + KH, kk), ID_MNMN, 1);
+                }
+                if (!(ok = mbar_wait(&bars[B_VFULL], i & 1, abort_word, a.flags))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t acc = (i > 0 || kk > 0);
                     mma_bf16(tP, mnmajor_desc(sb + AH, kk), mnmajor_desc(sb + VT, kk), ID_MNMN, acc);
                     mma_bf16(tP, mnmajor_desc(sb + AL, kk), mnmajor_desc(sb + VT, kk), ID_MNMN, 1);
                 }
@@ -690,15 +267,16 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
             const int tok = t_begin + i * kTile + r;
             const bool valid = tok < t_end;
             const float bl = valid ? a.beta_logits[(size_t)bh * T + tok] : 0.f;
-            bool w_ok = ok && mbar_wait(&bars[B_KTFULL], i & 1, abort_word, a.flags);
-            if (i > 0) w_ok = w_ok && mbar_wait(&bars[B_OPSFREE], (i - 1) & 1, abort_word, a.flags);
-            w_ok = __all_sync(0xffffffffu, w_ok);
+            bool w_ok = __all_sync(0xffffffffu,
+                                   ok && mbar_wait(&bars[B_KTFULL + (i & 1)], (i >> 1) & 1, abort_word, a.flags));
             float ssh = 0.f;
             if (w_ok) {
                 tc_fence_after();
-                tmem_ld32(tKT + lrow + half * 64, x);
-                tmem_ld32(tKT + lrow + half * 64 + 32, x + 32);
+                tmem_ld32(tKT(i) + lrow + half * 64, x);
+                tmem_ld32(tKT(i) + lrow + half * 64 + 32, x + 32);
                 tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&bars[B_KTREAD + (i & 1)]);  // K~(i+2) may overwrite this buffer
                 float ss8[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) ss8[k] = 0.f;
@@ -711,6 +289,9 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
             named_bar_sync(pair_bar, 64);
             ok = __all_sync(0xffffffffu, w_ok && xok[(s * 2 + (half ^ 1)) * 128 + r]);
             if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
+            // the operand tiles are free once the previous tile's products have read them
+            if (i > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_OPSFREE], (i - 1) & 1, abort_word, a.flags));
+            if (!ok) continue;
             const float ss = xss[(s * 2 + 0) * 128 + r] + xss[(s * 2 + 1) * 128 + r];
             const float inv = valid ? 1.0f / sqrtf(ss + a.l2_eps) : 0.f;
             const float beta = valid ? sigmoidf_(bl) : 0.f;
@@ -934,6 +515,140 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     // when launched as a programmatic dependent of the attention kernel, complete
     // only after it: later work in the stream stays ordered after both
     pdl_wait_primary();
+}
+
+// ============================================================== prep: W = phi_q^T S_{N-1}
+// The inter-frame read O_inter = Q' S_{N-1} = (Q phi_q^T) S_{N-1} is regrouped as
+// Q W with W = phi_q^T S_{N-1} (exact), so the attention kernel multiplies each
+// query tile by one d x d matrix.  One CTA per (batch, head), 8 warps:
+// phi_q arrives by TMA as an MN-major A operand (A[i][o] = phi_q[o][i]),
+// S_{N-1} by one bulk copy; the warps split S into bf16 hi + lo MN-major B tiles,
+// one thread issues W = phi_q^T S_hi + phi_q^T S_lo (16 MMAs, fp32 in TMEM), and
+// the warps write W (times the inter-frame gain c of a weighted pass) back as
+// the row-major bf16 hi + lo pair the attention kernel loads.
+namespace prep {
+constexpr uint32_t PHI = 0;
+constexpr uint32_t SF = PHI + kTileBytes;          // S_{N-1} fp32 [128][128]
+constexpr uint32_t SH = SF + 128 * 128 * 4;
+constexpr uint32_t SL = SH + kTileBytes;
+constexpr uint32_t BAR = SL + kTileBytes;          // 163,840
+constexpr uint32_t SMEM = BAR + 64;
+constexpr int kThreads = 256;
+enum { B_PHI = 0, B_S, B_MMA, B_COUNT };
+}  // namespace prep
+
+__global__ void __launch_bounds__(prep::kThreads, 1)
+    prep_tc_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_phiq) {
+    using namespace prep;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
+        return;
+    }
+    const uint32_t sb = smem_u32(smem);
+    uint64_t* bars = (uint64_t*)(smem + BAR);
+    uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
+    volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * a.H + h;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], 1);
+        *abort_word = 0;
+        fence_mbar_init();
+        fence_async_smem();
+        mbar_expect_tx(&bars[B_PHI], kTileBytes);
+        tma_load_3d(sb + PHI, &tm_phiq, &bars[B_PHI], 0, 0, h);
+        tma_load_3d(sb + PHI + kHalf, &tm_phiq, &bars[B_PHI], 64, 0, h);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 128);
+    // launched as a programmatic dependent: the previous kernel of the stream may
+    // write the state, so wait for it before reading S_{N-1}
+    pdl_wait_primary();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(&bars[B_S], 128 * 128 * 4);
+        bulk_load(sb + SF, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_S]);
+    }
+    const bool s_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_S], 0, abort_word, a.flags, a.wait_ns));
+    // S_{N-1} is in shared memory: only now may the attention kernel start, and
+    // through it the delta update that overwrites the state in place
+    __syncthreads();
+    pdl_launch_dependents();
+    const int half = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    if (s_ok) {
+        // S row `row`, columns 64 half..+63: bf16 hi + lo into the MN-major B tiles
+        const float4* Sp4 = reinterpret_cast<const float4*>(smem + SF) + row * 32 + half * 16;
+#pragma unroll
+        for (int k0 = 0; k0 < 16; ++k0) {
+            const int k = (k0 + lane) & 15;
+            const float4 v = Sp4[k];
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+            const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+            const uint2 hi = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
+                                        *reinterpret_cast<const uint32_t*>(&h23));
+            const uint2 lo = make_uint2(pack_bf16(v.x - __low2float(h01), v.y - __high2float(h01)),
+                                        pack_bf16(v.z - __low2float(h23), v.w - __high2float(h23)));
+            const uint32_t off = half * kHalf + sw128_offset(row, k >> 1) + (k & 1) * 8;
+            *reinterpret_cast<uint2*>(smem + SH + off) = hi;
+            *reinterpret_cast<uint2*>(smem + SL + off) = lo;
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        if (s_ok && mbar_wait(&bars[B_PHI], 0, abort_word, a.flags, a.wait_ns)) {
+            constexpr uint32_t ID_MNMN = idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16(tmem, mnmajor_desc(sb + PHI, kk), mnmajor_desc(sb + SH, kk), ID_MNMN, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16(tmem, mnmajor_desc(sb + PHI, kk), mnmajor_desc(sb + SL, kk), ID_MNMN, 1);
+        }
+        mma_commit(&bars[B_MMA]);  // also when nothing was issued: the waiters below return
+    }
+    bool m_ok = __all_sync(0xffffffffu, s_ok && mbar_wait(&bars[B_MMA], 0, abort_word, a.flags, a.wait_ns));
+    __syncthreads();
+    m_ok = m_ok && *abort_word == 0;  // thread 0's wait for phi_q may have failed
+    if (m_ok) {
+        tc_fence_after();
+        // W row `row` (TMEM lane), columns 64 half..+63 -> bf16 hi + lo, row-major
+        const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+        const float cg = a.mix ? a.mix[bh * 2 + 1] : 1.0f;
+        const size_t base = ((size_t)bh * 128 + row) * 128 + half * 64;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float x[32];
+            tmem_ld32(tmem + lrow + half * 64 + c * 32, x);
+            tmem_ld_wait();
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float w0 = x[2 * q] * cg, w1 = x[2 * q + 1] * cg;
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(w0, w1);
+                hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
+                lo[q] = pack_bf16(w0 - __low2float(hv), w1 - __high2float(hv));
+            }
+            uint4* dh = reinterpret_cast<uint4*>(a.WT_hi + base + c * 32);
+            uint4* dl = reinterpret_cast<uint4*>(a.WT_lo + base + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                dh[q] = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+                dl[q] = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 }  // namespace tc

@@ -162,6 +162,32 @@ hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc,
                                     const float* gate_logits, const float* beta_logits,
                                     float* state, int clean_pass, void* out, void* stream);
 
+/* hyb_attn_forward_token_level -- the token-level access variant of a pass
+ * (ARL2 summary §4, ablations: token-level against frame-level access to the
+ * memory).  The pages give it no formulas; the reading taken: on a clean pass
+ * the tokens of the frame update the state one after another by the
+ * frame-level rule applied to a single token, with a per-token forget gate,
+ *     S_t = alpha_t S_{t-1} + beta_t k'_t (v'_t - k'_t^T S_{t-1}),
+ *     alpha_t = sigmoid(gate_logit_t), beta_t = sigmoid(beta_logit_t),
+ * and token t reads the state before its own update, O_inter[t] = q'_t S_{t-1}
+ * (causal within the frame).  The residual is taken against the undecayed
+ * state, as in the frame-level rule, so a one-token frame gives the same update
+ * under both accesses (this is not the decayed residual of "Gated Delta
+ * Networks").  out = O_intra + O_inter, rounded once; state holds S_{N-1} on
+ * entry and the state after the frame's last token on return.  A query-only
+ * pass (clean_pass = 0) is exactly hyb_attn_forward's.  Computed in chunks of
+ * 64 tokens in fp32 with only relative decays exp(Lambda_a - Lambda_b) <= 1.
+ * Same arguments, layouts, alignment and errors as hyb_attn_forward, except the
+ * workspace: at least hyb_attn_token_level_workspace_bytes(desc) bytes
+ * (HYB_ERR_WORKSPACE otherwise), zero-filled once like hyb_attn_forward's. */
+size_t hyb_attn_token_level_workspace_bytes(const hyb_attn_desc* desc);
+hyb_status hyb_attn_forward_token_level(const hyb_attn_desc* desc,
+                                        const void* q, const void* k, const void* v,
+                                        const void* phi_q, const void* phi_k, const void* phi_v,
+                                        const float* gate_logits, const float* beta_logits,
+                                        float* state, int clean_pass, void* out,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* hyb_kvcache_attn_forward -- the softmax baseline the hybrid layer replaces
  * (ARL2 summary §1, problem statement: softmax self-attention whose key/value
  * cache grows with every generated chunk; §4, the memory and wall-clock
@@ -194,6 +220,20 @@ hyb_status hyb_kvcache_attn_forward(const hyb_attn_desc* desc, const void* q, co
  * read, else HYB_OK (or HYB_ERR_CUDA if the synchronisation failed). */
 hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
 
+/* ---- fault test (tests only) --------------------------------------------------
+ * Process-wide and off by default; affects calls made after it, on any device.
+ * wait_limit_us > 0 replaces the 2 s limit of the attention kernel's bounded
+ * device waits (mbarrier waits) by that many microseconds (at most 10 s);
+ * 0 restores 2 s.  skip_v_loads = 1 makes the attention kernel's value-tile
+ * producer issue no loads at all, so the first wait for a value tile expires:
+ * the kernel then sets the TIMEOUT flag that hyb_attn_get_device_status reports
+ * as HYB_ERR_TIMEOUT, stores no output, waits for the products it has issued,
+ * frees its tensor memory and returns, leaving the device usable.  No copy is
+ * in flight when the wait expires.  The delta update is not affected.
+ * HYB_ERR_INVALID for skip_v_loads outside {0, 1} or a limit above 10 s.
+ * Not thread-safe; set it back to (0, 0) after the test. */
+hyb_status hyb_attn_set_fault_test(int skip_v_loads, unsigned wait_limit_us);
+
 /* ---- optional kernel timing (benchmarks) ------------------------------------
  * Process-wide and off by default.  hyb_attn_timing_begin(n) creates 2n CUDA
  * events on the current device; until hyb_attn_timing_end, every kernel that
@@ -203,7 +243,7 @@ hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
  * stream is being captured into a CUDA graph.  hyb_attn_timing_end waits for
  * the recorded events, sums each kernel's launch count and event time into
  * *out, destroys the events and turns timing off.  Not thread-safe. */
-#define HYB_NUM_KERNELS 4
+#define HYB_NUM_KERNELS 7
 typedef struct {
     int launches[HYB_NUM_KERNELS];     /* indexed as hyb_attn_kernel_name() */
     double total_ms[HYB_NUM_KERNELS];
@@ -213,7 +253,9 @@ typedef struct {
 hyb_status hyb_attn_timing_begin(int max_launches);
 hyb_status hyb_attn_timing_end(hyb_attn_timing* out);
 /* "prep", "intra_frame_attention", "delta_update" (bf16: the whole update; fp32:
- * its token-split reduction), "delta_update_apply" (fp32 only); NULL if out of range */
+ * its token-split reduction), "delta_update_apply" (fp32 only), and the three
+ * kernels of a token-level clean pass: "token_chunk_prep", "token_chain",
+ * "token_reads"; NULL if out of range */
 const char* hyb_attn_kernel_name(int kernel);
 
 /* Static string naming a status code. */
