@@ -54,12 +54,7 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     const int BH = d->B * d->H;
     const int ntiles = (d->T + kUpdateTile - 1) / kUpdateTile;
     int want = bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH;
-    if (bf16) {
-        // the update runs beside the attention kernel (two query tiles per CTA):
-        // size its clusters to the SMs that grid leaves free, when it leaves some
-        const long attn_ctas = (long)((ntiles + 1) / 2) * BH;
-        if (attn_ctas < kNumSMs && (kNumSMs - attn_ctas) / BH >= 2) want = (int)((kNumSMs - attn_ctas) / BH);
-    }
+
     if (bf16 && want > tc::kMaxClusterRanks) want = tc::kMaxClusterRanks;
     if (want > ntiles) want = ntiles;
     if (want < 1) want = 1;
@@ -132,8 +127,8 @@ cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
     return e;
 }
 
-// CTAs of the attention kernel along the query axis: two 128-query tiles each.
-unsigned attn_pairs(int T) { return (unsigned)(((T + tc::kTile - 1) / tc::kTile + 1) / 2); }
+// CTAs of the attention kernel along the query axis: one per 128-query tile.
+unsigned attn_tiles(int T) { return (unsigned)((T + tc::kTile - 1) / tc::kTile); }
 
 template <int D, typename TIO>
 cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
@@ -236,7 +231,7 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     constexpr int D = 128;
     cudaError_t e;
     if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return e;
+    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
     if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
     const uint64_t row_bytes = (uint64_t)a.H * D * 2;
     const uint64_t bh = (uint64_t)a.B * a.H;
@@ -268,13 +263,13 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (le != cudaSuccess) return le;
     cudaLaunchConfig_t acfg = {};
-    acfg.gridDim = dim3(attn_pairs(a.T), a.H, a.B);
-    acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
-    acfg.dynamicSmemBytes = tc::pp::SMEM;
+    acfg.gridDim = dim3(attn_tiles(a.T), a.H, a.B);
+    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::attn::SMEM;
     acfg.stream = st;
     acfg.attrs = pdl;
     acfg.numAttrs = 1;
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tw, tout); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw, tout); });
     if (e != cudaSuccess) return e;
     if (le != cudaSuccess) return le;
     if (clean) {
@@ -407,7 +402,7 @@ cudaError_t launch_token_level(LayerArgs a, const TokPlan& tp, char* ws, cudaStr
     a.oi_ext = oi;
     if constexpr (D == 128) {
         static unsigned char done_attn[kMaxDevices];
-        if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
         const uint64_t row_bytes = (uint64_t)a.H * D * 2;
         CUtensorMap tq, tk, tv, tout;
         if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
@@ -417,14 +412,14 @@ cudaError_t launch_token_level(LayerArgs a, const TokPlan& tp, char* ws, cudaStr
             return cudaErrorInvalidValue;
         if (!a.out) tout = tq;
         cudaLaunchConfig_t acfg = {};
-        acfg.gridDim = dim3(attn_pairs(a.T), a.H, a.B);
-        acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
-        acfg.dynamicSmemBytes = tc::pp::SMEM;
+        acfg.gridDim = dim3(attn_tiles(a.T), a.H, a.B);
+        acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+        acfg.dynamicSmemBytes = tc::attn::SMEM;
         acfg.stream = st;
         cudaError_t le = cudaSuccess;
         // tq stands in for the unused W map
         e = timed(K_ATTN, st,
-                  [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tq, tout); });
+                  [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
         if (e != cudaSuccess) return e;
         if (le != cudaSuccess) return le;
     } else {
@@ -516,7 +511,7 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
 
     static unsigned char done_attn[kMaxDevices];
     cudaError_t e;
-    if ((e = opt_in_smem(tc::attention_pp_kernel, tc::pp::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
+    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
     const uint64_t row_bytes = (uint64_t)H * D * 2;
     CUtensorMap tq, tk, tv, tout;
     if (!map3d(&tq, q, (uint64_t)H * D, T, B, row_bytes, row_bytes * T) ||
@@ -525,13 +520,13 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
         !map3d(&tout, out, (uint64_t)H * D, T, B, row_bytes, row_bytes * T))
         return HYB_ERR_CUDA;
     cudaLaunchConfig_t acfg = {};
-    acfg.gridDim = dim3(attn_pairs(T), H, B);
-    acfg.blockDim = dim3(tc::pp::kThreads, 1, 1);
-    acfg.dynamicSmemBytes = tc::pp::SMEM;
+    acfg.gridDim = dim3(attn_tiles(T), H, B);
+    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+    acfg.dynamicSmemBytes = tc::attn::SMEM;
     acfg.stream = st;
     cudaError_t le = cudaSuccess;
     // tq stands in for the unused W map
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_pp_kernel, a, tq, tk, tv, tq, tout); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
     if (e != cudaSuccess || le != cudaSuccess) return HYB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }

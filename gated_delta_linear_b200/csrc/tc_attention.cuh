@@ -8,176 +8,131 @@
 // every token reads the same pre-update state).  The layer output is
 // O_intra + O_inter (the pages leave the combination open; this library sums).
 //
-// One CTA takes two 128-query tiles (A and B) of one (batch, head) and streams
-// the frame's keys and values past both in 128-key blocks:
-//   warps 0-3   softmax of tile A, one query row (TMEM lane) per thread;
-//   warps 4-7   softmax of tile B;
-//   warp 8      TMA producer of Q_A, Q_B, the K ring and, at the end, W;
-//   warp 9      the single tcgen05 MMA issuer;
-//   warp 10     TMA producer of the V ring.
-// The two tiles ping-pong: while the softmax warps of one tile turn its scores
-// into probabilities on the MUFU pipe, the tensor pipe runs the other tile's
-// O += P V and its next S = Q K^T, so neither pipe waits for the other.
-//
-// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
-// P_t (bf16 pairs, the A operand of O_t += P_t V) is written over the first 64
-// columns of S_t once the scores are in registers.  MMAs into different
-// accumulators are not ordered by the hardware, so S_t(j+1) is issued only
-// after O_t += P_t(j) V_j has completed.
-//
-// Softmax offset: probabilities are 2^(s x - m) with a per-row offset m (the
-// first block's row max, in log2 units) that moves only when a block's row sum
-// leaves [0, 2^63): then the block is redone against the row's max and O, l
-// are rescaled (O_t is idle then: S_t(j) is issued after P_t(j-1) V has
-// completed).  The offset cancels in O / l, so this is the same softmax.
-//
-// Epilogue: after the last block each tile's S buffer is free, and O_inter = Q_t W_hi + Q_t W_lo (W = phi_q^T S_{N-1}, a two-term
-// bf16 split written by the prep kernel, loaded into K stages the last score
-// products have freed) is computed there; out = a O_t / l + O_inter is rounded
-// once to bf16, staged in the tile's Q buffer and written with TMA stores.
+// attention_kernel: one CTA per (128-query tile, head, batch), 11 warps.
+// Warp 8 streams Q and the K ring, warp 10 the V ring, with TMA into
+// 128B-swizzled shared memory; warp 9 issues the tcgen05 MMAs; warps 0-7 run
+// the online softmax, a query row per pair of threads (warps w and w+4, 64
+// scores each in registers).  Near the end of the key loop the Q tile is
+// multiplied by W = phi_q^T S_{N-1} (a two-term bf16 split W_hi + W_lo, row
+// major: an MN-major B operand), so the inter-frame read lands in TMEM next to
+// the softmax accumulator and the epilogue writes out = O_intra + O_inter once.
+//   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
+//                 [384,448) Q, [448,512) P (bf16, two per 32-bit column: the
+//                 A operands of S = Q K^T and O += P V).  Q is copied from
+//                 shared memory into TMEM once; as soon as the softmax has S_j
+//                 in registers the MMA warp issues S_{j+2} into its buffer, so
+//                 scores run a tile ahead of the softmax, and the softmax loads
+//                 S_{j+1} while it hands P_j over.  With both MMA A operands in
+//                 TMEM only the B operand (K or V) is read from shared memory.
+//   Softmax: exponents against a running offset (the first tile's row max),
+//                 moved only when a tile's partial sum over a half row leaves
+//                 [0, 2^63); all exponentials on the MUFU pipe.
+//   Shared memory: Q 32 KB | K 3 x 32 KB | V 3 x 32 KB.  Near the end W_hi
+//                 and W_lo take the K stages of key tiles n-3 and n-2 (unused
+//                 stages when n < 3) and O_inter = Q W_hi + Q W_lo goes to the
+//                 S buffer the last tile does not use while the softmax works
+//                 on the last two tiles; the bf16 output tile is assembled in
+//                 the Q buffer and written with two TMA stores.
+//   Token-level access (a.oi_ext): no W product; the epilogue adds the fp32
+//                 read the token-level kernels computed.
+//   Every CTA signals at entry that the next kernel (the delta update, which
+//   reads none of this kernel's outputs) may start on idle SMs.
 #pragma once
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
+#include "tc_kernels.cuh"
 
 namespace hyb {
 namespace tc {
 
 using namespace sm100;
 
-namespace pp {
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
-constexpr uint32_t QA = 0;
-constexpr uint32_t QB = QA + kTileBytes;
-constexpr uint32_t K0 = QB + kTileBytes;
+namespace attn {
+constexpr int kKStages = 3;                    // K ring depth
+constexpr int kVStages = 3;                    // V ring depth
+constexpr uint32_t Q = 0;
+constexpr uint32_t K0 = Q + kTileBytes;
 constexpr uint32_t V0 = K0 + kKStages * kTileBytes;
-constexpr uint32_t BAR = V0 + kVStages * kTileBytes;   // 229,376
-constexpr uint32_t SMEM = BAR + 256;                    // 229,632 B
-constexpr int kThreads = 352;  // 11 warps: up to 184 registers per thread
+constexpr uint32_t BAR = V0 + kVStages * kTileBytes;
+constexpr uint32_t XCH = BAR + 256;            // softmax pair exchange: [2 parity][2 halves][128 rows] floats
+constexpr uint32_t XFL = XCH + 2048;           // and codes [2][2][128] bytes
+constexpr uint32_t SMEM = XFL + 512;           // 232,192 B
+constexpr int kSoftmaxThreads = 256;           // warps 0-7: rows 32(w&3)..+31, column half w>>2
 constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadVWarp = 10;
-enum {
-    B_QA = 0, B_QB = 1, B_W = 2, B_KFULL = 3, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
-    B_VEMPTY = B_VFULL + kVStages, B_SFULL = B_VEMPTY + kVStages, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-    B_OIDONE = B_PVDONE + 2, B_DRAIN = B_OIDONE + 2, B_TURN = B_DRAIN + 1, B_COUNT = B_TURN + 2
-};
-static_assert(B_COUNT * 8 + 16 <= 256, "barrier block");
-static_assert(SMEM <= 232448, "shared memory per CTA");
-}  // namespace pp
+constexpr int kThreads = 352;
+enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12, B_SFULL = 15,
+       B_SREAD = 17, B_QTM = 19, B_PFULL = 20, B_PVDONE = 21, B_COUNT = 22 };
+static_assert(B_COUNT * 8 + 8 <= 256, "barrier block");
+}  // namespace attn
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
-    uint32_t r[8];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-        : "memory");
-}
-
-// Named barrier over `count` threads that also returns the AND of `pred` over them.
-__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\n"
-        "barrier.cta.red.and.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
-}
-
-// p = 2^(x * scale + neg_m) for the 128 scores of a row, written as bf16 pairs
-// (round to nearest) over TMEM columns [0, 64) of the row's S buffer; returns
-// the row sum of p in fp32.
-__device__ __forceinline__ float exp_row_to_tmem(const float* x, float scale, float neg_m, uint32_t tP) {
+// p = 2^(x * scale + neg_m) for N scores, as N/2 bf16 pairs (round to
+// nearest) in pk; returns the sum of p in fp32 (the exponentials on the MUFU
+// pipe, the pair conversion one instruction per two values).
+template <int N>
+__device__ __forceinline__ float exp_scores(const float* x, float scale, float neg_m, uint32_t* pk) {
     float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float e0 = ex2(fmaf(x[16 * c + 2 * k], scale, neg_m));
-            const float e1 = ex2(fmaf(x[16 * c + 2 * k + 1], scale, neg_m));
-            l4[(2 * k) & 3] += e0;
-            l4[(2 * k + 1) & 3] += e1;
-            pk[k] = pack_bf16(e0, e1);
-        }
-        tmem_st8u(tP + 8 * c, pk);
+    for (int k = 0; k < N / 2; ++k) {
+        const float e0 = ex2(fmaf(x[2 * k], scale, neg_m));
+        const float e1 = ex2(fmaf(x[2 * k + 1], scale, neg_m));
+        l4[(2 * k) & 3] += e0;
+        l4[(2 * k + 1) & 3] += e1;
+        pk[k] = pack_bf16(e0, e1);
     }
     return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
-__global__ void __launch_bounds__(pp::kThreads, 1)
-    attention_pp_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_q,
-                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
-    using namespace pp;
+__global__ void __launch_bounds__(attn::kThreads, 1)
+    attention_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o) {
+    using namespace attn;
     extern __shared__ __align__(1024) uint8_t smem[];
-    // 128B-swizzled tiles need a 1024-byte aligned base: report and leave if not
+    // 128B-swizzled tiles need a 1024-byte aligned base (the dynamic window starts
+    // after the 1 KB reserved block); report and leave if it is not
     if (smem_u32(smem) & 1023u) {
         if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
         return;
     }
-    // the delta update of this pass reads nothing this kernel writes: it may
-    // start on SMs this grid leaves idle
+    // the delta update of this pass does not read anything this kernel writes:
+    // it may start on SMs this grid leaves idle
     pdl_launch_dependents();
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
     volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+    volatile int* epi_bad = (volatile int*)(tmem_slot + 2);  // a softmax warp missed its epilogue
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T;
-    const int nq = (T + kTile - 1) / kTile;
-    const int qtA = 2 * blockIdx.x;
-    const bool hasB = qtA + 1 < nq;
-    const int n = (a.T_kv + kTile - 1) / kTile;  // key blocks
-    const bool inter = a.inter != 0;
+    const int q0 = qt_ * kTile;
+    const int n = (a.T_kv + kTile - 1) / kTile;  // key tiles
+    const bool inter = a.inter != 0;             // add O_inter = Q W (hybrid layer)
     const int bh = b * a.H + h;
-    const int xh = h * 128;
-    // K stages that receive W_hi / W_lo at the end (free once the score products
-    // of key blocks n-3 / n-2 have completed; stages no block uses when n is small)
+    // K stages that receive W_hi / W_lo at the end (free once the scores of key
+    // tiles n-3 / n-2 are computed; stages no tile uses when n is small)
     const int wst_hi = n >= 3 ? (n - 3) % kKStages : 2;
     const int wst_lo = n >= 2 ? (n - 2) % kKStages : 1;
 
     if (threadIdx.x == kLoadWarp * 32) {
-        // the producer initialises the barriers and starts the first loads before
-        // the block synchronises (the loads land on its own barriers)
+        // the producer initialises the barriers and starts the first loads
+        // before the block synchronises (the loads land on its own barriers)
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1 || i == B_TURN || i == B_TURN + 1) ? 128 : 1);
+            mbar_init(&bars[i],
+                      (i == B_PFULL || i == B_QTM || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads : 1);
         *abort_word = 0;
+        *epi_bad = 0;
         fence_mbar_init();
         fence_async_smem();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        mbar_expect_tx(&bars[B_QA], kTileBytes);
-        tma_load_3d(sb + QA, &tm_q, &bars[B_QA], xh, qtA * kTile, b);
-        tma_load_3d(sb + QA + kHalf, &tm_q, &bars[B_QA], xh + 64, qtA * kTile, b);
-        mbar_expect_tx(&bars[B_KFULL], kTileBytes);
-        tma_load_3d(sb + K0, &tm_k, &bars[B_KFULL], xh, 0, b);
-        tma_load_3d(sb + K0 + kHalf, &tm_k, &bars[B_KFULL], xh + 64, 0, b);
-        if (hasB) {
-            mbar_expect_tx(&bars[B_QB], kTileBytes);
-            tma_load_3d(sb + QB, &tm_q, &bars[B_QB], xh, (qtA + 1) * kTile, b);
-            tma_load_3d(sb + QB + kHalf, &tm_q, &bars[B_QB], xh + 64, (qtA + 1) * kTile, b);
-        }
-        for (int j = 1; j < kKStages && j < n; ++j) {
+        const int xh = h * 128;
+        mbar_expect_tx(&bars[B_Q], kTileBytes);
+        tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0, b);
+        tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
+        for (int j = 0; j < kKStages && j < n; ++j) {
             mbar_expect_tx(&bars[B_KFULL + j], kTileBytes);
             tma_load_3d(sb + K0 + j * kTileBytes, &tm_k, &bars[B_KFULL + j], xh, j * kTile, b);
             tma_load_3d(sb + K0 + j * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + j], xh + 64, j * kTile, b);
@@ -188,11 +143,16 @@ __global__ void __launch_bounds__(pp::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // S buffers 0 / 1, O, Q and P as bf16 pairs (the A operands of the score
+    // and value products)
+    const uint32_t tS0 = tmem, tO = tmem + 256, tQ = tmem + 384, tP = tmem + 448;
+    const uint32_t tOI = tS0 + (n & 1) * 128;  // the S buffer the last tile does not use
 
     if (warp == kLoadVWarp) {
         // ------------------------------------------------ TMA producer: V ring
         if (lane == 0) {
             tma_prefetch_desc(&tm_v);
+            const int xh = h * 128;
             // (a fault test may switch this producer off: the MMA issuer's wait for V
             // then expires, and the kernel reports a timeout and unwinds)
             for (int j = 0; j < n && !a.dbg_skip_v; ++j) {
@@ -207,17 +167,21 @@ __global__ void __launch_bounds__(pp::kThreads, 1)
         }
         __syncwarp();
     } else if (warp == kLoadWarp) {
-        // ------------------------------------------------ TMA producer: K ring, then W
+        // ------------------------------------------------ TMA producer: Q, K ring, W
+        // (its own warp, so K tiles run ahead of the V ring's waits)
         if (lane == 0) {
             tma_prefetch_desc(&tm_w);
+            const int xh = h * 128;
             bool ok = true;
-            for (int j = kKStages; j < n && ok; ++j) {
+            for (int j = kKStages; j < n && ok; ++j) {  // Q and K_0..K_2 were issued at entry
                 const int ks = j % kKStages;
                 if (!(ok = mbar_wait(&bars[B_KEMPTY + ks], ((j / kKStages) + 1) & 1, abort_word, a.flags, a.wait_ns))) break;
                 mbar_expect_tx(&bars[B_KFULL + ks], kTileBytes);
                 tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, j * kTile, b);
                 tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64, j * kTile, b);
             }
+            // W_hi / W_lo (row-major, MN-major operands) into K stages freed by S_{n-3} / S_{n-2}
+            const int nbh = a.B * a.H;
             if (inter && ok && n >= 3)
                 ok = mbar_wait(&bars[B_KEMPTY + wst_hi], ((n - 3) / kKStages) & 1, abort_word, a.flags, a.wait_ns);
             if (inter && ok && n >= 2)
@@ -226,7 +190,6 @@ __global__ void __launch_bounds__(pp::kThreads, 1)
             // grid starts (programmatic dependent launch): wait for it here
             if (inter) pdl_wait_primary();
             if (inter && ok) {
-                const int nbh = a.B * a.H;
                 mbar_expect_tx(&bars[B_W], 2 * kTileBytes);
                 tma_load_3d(sb + K0 + wst_hi * kTileBytes, &tm_w, &bars[B_W], 0, 0, bh);
                 tma_load_3d(sb + K0 + wst_hi * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
@@ -237,218 +200,286 @@ __global__ void __launch_bounds__(pp::kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
+        // S_j = Q K_j^T into S buffer j&1 (A = Q from TMEM); S_{j+2} reuses the
+        // buffer as soon as the softmax has S_j in registers, so scores run a
+        // tile ahead.  O += P_j V_j once P_j is in TMEM.
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
-            const int ntile = hasB ? 2 : 1;
-            // S_t(0) = Q_t K_0^T
-            if (!(mbar_wait(&bars[B_KFULL], 0, abort_word, a.flags, a.wait_ns))) goto drain;
-            for (int t = 0; t < ntile; ++t) {
-                if (!(mbar_wait(&bars[B_QA + t], 0, abort_word, a.flags, a.wait_ns))) goto drain;
+            // S_0 and S_1 take Q from shared memory (no wait for its copy into TMEM)
+            bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns);
+            bool q_in_tmem = false;
+            for (int j = 0; j < 2 && j < n && ok; ++j) {
+                if (!(ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags, a.wait_ns))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem + t * 128, kmajor_desc(sb + QA + t * kTileBytes, kk), kmajor_desc(sb + K0, kk),
-                             ID_KK, kk > 0);
-                mma_commit(&bars[B_SFULL + t]);
+                    mma_bf16(tS0 + j * 128, kmajor_desc(sb + Q, kk), kmajor_desc(sb + K0 + j * kTileBytes, kk), ID_KK,
+                             kk > 0);
+                mma_commit(&bars[B_SFULL + j]);
+                mma_commit(&bars[B_KEMPTY + j]);
             }
-            mma_commit(&bars[B_KEMPTY]);
-            for (int j = 0; j < n; ++j) {
+            for (int j = 0; j < n && ok; ++j) {
+                const int sbuf = j & 1;
+                if (j + 2 < n) {
+                    const int ks = (j + 2) % kKStages;
+                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags, a.wait_ns))) break;
+                    if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags, a.wait_ns))) break;
+                    if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags, a.wait_ns))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tS0 + sbuf * 128, tQ + kk * 8, kmajor_desc(sb + K0 + ks * kTileBytes, kk), ID_KK,
+                                    kk > 0);
+                    mma_commit(&bars[B_SFULL + sbuf]);
+                    mma_commit(&bars[B_KEMPTY + ks]);
+                }
+                if (inter && j == (n >= 2 ? n - 2 : 0)) {
+                    // O_inter = Q W_hi + Q W_lo into S buffer n&1 (free once the
+                    // softmax has S_{n-2} in registers; unused when n == 1), run
+                    // while the softmax works on the last two tiles
+                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags, a.wait_ns))) break;
+                    if (n >= 2 &&
+                        !(ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags, a.wait_ns)))
+                        break;
+                    if (!(ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags, a.wait_ns))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
+                    mma_commit(&bars[B_OIDONE]);
+                }
                 const int vs = j % kVStages;
-                const int ks1 = (j + 1) % kKStages;
-                for (int t = 0; t < ntile; ++t) {
-                    // O_t += P_t(j) V_j (P_t in TMEM over the first columns of S_t)
-                    if (!(mbar_wait(&bars[B_PFULL + t], j & 1, abort_word, a.flags, a.wait_ns))) goto drain;
-                    if (t == 0 && !(mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags, a.wait_ns)))
-                        goto drain;
-                    tc_fence_after();
+                if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags, a.wait_ns))) break;
+                if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags, a.wait_ns))) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                                    mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
-                    mma_commit(&bars[B_PVDONE + t]);
-                    if (t == ntile - 1) mma_commit(&bars[B_VEMPTY + vs]);
-                    if (j + 1 < n) {
-                        // S_t(j+1) = Q_t K_{j+1}^T into S_t, once P_t(j) has been read
-                        if (t == 0 &&
-                            !(mbar_wait(&bars[B_KFULL + ks1], ((j + 1) / kKStages) & 1, abort_word, a.flags, a.wait_ns)))
-                            goto drain;
-                        if (!(mbar_wait(&bars[B_PVDONE + t], j & 1, abort_word, a.flags, a.wait_ns))) goto drain;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_bf16(tmem + t * 128, kmajor_desc(sb + QA + t * kTileBytes, kk),
-                                     kmajor_desc(sb + K0 + ks1 * kTileBytes, kk), ID_KK, kk > 0);
-                        mma_commit(&bars[B_SFULL + t]);
-                        if (t == ntile - 1) mma_commit(&bars[B_KEMPTY + ks1]);
-                    }
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tO, tP + kk * 8, mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
+                mma_commit(&bars[B_PVDONE]);
+                mma_commit(&bars[B_VEMPTY + vs]);
             }
-            // O_inter_t = Q_t W_hi + Q_t W_lo into S_t (free once P_t(n-1) V has completed)
-            if (inter && !(mbar_wait(&bars[B_W], 0, abort_word, a.flags, a.wait_ns))) goto drain;
-            for (int t = 0; t < ntile; ++t) {
-                if (inter) {
-                    if (!(mbar_wait(&bars[B_PVDONE + t], (n - 1) & 1, abort_word, a.flags, a.wait_ns))) goto drain;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + t * 128, kmajor_desc(sb + QA + t * kTileBytes, kk),
-                                 mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + t * 128, kmajor_desc(sb + QA + t * kTileBytes, kk),
-                                 mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
-                }
-                mma_commit(&bars[B_OIDONE + t]);
-            }
-        drain:
-            // (a failed wait has already set the abort word and the TIMEOUT flag)
-            // every MMA issued so far completes before TMEM is released
-            mma_commit(&bars[B_DRAIN]);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(smem_u32(&bars[B_DRAIN]), 0) && globaltimer_ns() - t0 < a.wait_ns) {
+            // drain: every MMA issued so far completes before TMEM is released
+            mma_commit(&bars[B_Q]);
+            uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(smem_u32(&bars[B_Q]), 1) && globaltimer_ns() - t0 < a.wait_ns) {
             }
         }
         __syncwarp();
-    } else if (warp < 8) {
-        // ------------------------------------------------ softmax + epilogue of tile t
-        const int t = warp >> 2;
-        if (t == 0 || hasB) {
-            const int r = (warp & 3) * 32 + lane;
-            const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
-            const uint32_t tS = tmem + t * 128 + lrow;
-            const uint32_t tO = tmem + 256 + t * 128 + lrow;
-            const float scale = a.sm_scale_log2;
-            float m = 0.f, l = 0.f;
-            float x[128];
-            bool ok = true;
-            for (int j = 0; j < n; ++j) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + t], j & 1, abort_word, a.flags, a.wait_ns));
-                if (!ok) break;
-                tc_fence_after();
+    } else {
+        // ------------------------------------------------ softmax + epilogue
+        // Warps w and w+4 share query rows 32(w&3)..+31 (TMEM lanes); warp w>>2
+        // takes score and output columns 64(w>>2)..+63, so two softmax warps
+        // per SM sub-partition interleave their exponentials.  S_j is released
+        // (SREAD) as soon as it is in registers, so S_{j+2} is computed while
+        // this tile is exponentiated, and S_{j+1} is loaded before P_j is
+        // handed to the MMA warp.
+        //
+        // Offset: exponents are taken against a running offset m (log2 units)
+        // that is the row max of the first tile and moves only when a tile's
+        // partial sum over a half leaves [0, 2^63): the tile is then redone
+        // against the row's max and O, l are rescaled.  Every value stays
+        // finite, P <= 2^63, and the result is the same softmax (the offset
+        // cancels in O / l).
+        //
+        // The two warps of a pair exchange a code per row and tile (0: a wait
+        // failed, 1: ok, 2: offset too low) at their pair barrier and take the
+        // same path from it; a warp whose wait failed keeps arriving at the
+        // pair barriers to the end, so neither warp ever waits for the other
+        // without a partner.
+        const int g = warp & 3, hf = warp >> 2;
+        const int r = g * 32 + lane;
+        const int pair_bar = 1 + g;
+        const uint32_t lrow = (uint32_t)(g * 32) << 16;
+        const uint32_t cs = hf * 64;
+        float* xch = (float*)(smem + XCH);
+        uint8_t* xfl = smem + XFL;
+        const int mine = hf * 128 + r, theirs = (hf ^ 1) * 128 + r;  // + parity * 256
+        const float scale = a.sm_scale_log2;
+        float m = 0.f, l = 0.f;
+        float x[64];
+        // this half of Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns));
+        if (ok) {
+            uint32_t qv[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, x + 32 * c);
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hf * kHalf + sw128_offset(r, c));
+                qv[4 * c] = v.x;
+                qv[4 * c + 1] = v.y;
+                qv[4 * c + 2] = v.z;
+                qv[4 * c + 3] = v.w;
+            }
+            tmem_st32u(tQ + lrow + hf * 32, qv);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[B_QTM]);
+        }
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags, a.wait_ns));
+        if (ok) {
+            tc_fence_after();
+            tmem_ld32(tS0 + lrow + cs, x);
+            tmem_ld32(tS0 + lrow + cs + 32, x + 32);
+        }
+        for (int j = 0; j < n; ++j) {
+            const int s = j & 1;
+            const bool w_ok = ok;
+            uint32_t pk[32];
+            float lt = 0.f;
+            if (w_ok) {
                 tmem_ld_wait();
-                const int valid = a.T_kv - j * kTile;
-                if (valid < 128) {
+                tc_fence_before();
+                mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
+                const int valid = a.T_kv - j * kTile - (int)cs;
+                if (valid < 64) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
+                    for (int c = 0; c < 64; ++c)
                         if (c >= valid) x[c] = -INFINITY;
                 }
-                if (j == 0) m = row_max<128>(x) * scale;  // the first block's row max sets the offset
-                // the two tiles take turns on the MUFU pipe: tile B's exponentials of
-                // block j start after tile A's, tile A's of block j+1 after tile B's
-                // of block j, so each tile's products run while the other one exponentiates
-                if (hasB && (t == 1 || j > 0)) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_TURN + t], (t == 1 ? j : j - 1) & 1, abort_word,
-                                                           a.flags, a.wait_ns));
-                    if (!ok) break;
-                }
-                float lt = exp_row_to_tmem(x, scale, -m, tS);
-                const bool redo = !(lt < 9.2233720e18f);  // >= 2^63, inf or NaN
-                if (__any_sync(0xffffffffu, redo)) {
-                    // the offset is too low for this block (or a score is not finite):
-                    // move it to the row's max, rescale O and l, redo P_t(j)
-                    float f = 1.0f;
-                    if (redo) {
-                        const float mn = fmaxf(m, row_max<128>(x) * scale);
-                        f = ex2(m - mn);
-                        m = mn;
-                    }
-                    if (j > 0) {
-                        // (in 8-column pieces: the 128 scores stay live in registers)
-#pragma unroll 1
-                        for (int c = 0; c < 128; c += 8) {
-                            float o[8];
-                            uint32_t ou[8];
-                            tmem_ld8(tO + c, o);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) ou[q] = __float_as_uint(o[q] * f);
-                            tmem_st8u(tO + c, ou);
-                        }
-                    }
-                    l *= f;
-                    lt = exp_row_to_tmem(x, scale, -m, tS);
-                }
-                l += lt;
-                if (hasB && (t == 0 || j + 1 < n)) mbar_arrive(&bars[B_TURN + (t ^ 1)]);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[B_PFULL + t]);
             }
-            // epilogue: out = a O / l + O_inter, one bf16 rounding, through the Q buffer
-            const bool e_ok =
-                __all_sync(0xffffffffu, ok && mbar_wait(&bars[B_OIDONE + t], 0, abort_word, a.flags, a.wait_ns));
-            const int q0 = (qtA + t) * kTile;
-            const int tok = q0 + r;
-            if (e_ok) {
+            if (j == 0) {
+                // the first tile's row max over both halves sets the offset
+                const float hm = w_ok ? row_max<64>(x) : -INFINITY;
+                xch[mine] = hm;
+                named_bar_sync(pair_bar, 64);
+                m = fmaxf(hm, xch[theirs]) * scale;
+            }
+            bool redo_h = false;
+            if (w_ok) {
+                lt = exp_scores<64>(x, scale, -m, pk);
+                redo_h = !(lt < 9.2233720e18f);  // >= 2^63, inf or NaN
+            }
+            xfl[s * 256 + mine] = w_ok ? (redo_h ? 2 : 1) : 0;
+            named_bar_sync(pair_bar, 64);
+            const uint8_t pc = xfl[s * 256 + theirs];
+            ok = __all_sync(0xffffffffu, w_ok && pc != 0);  // the same in both warps of the pair
+            const bool redo = ok && (redo_h || pc == 2);
+            const bool any_redo = __any_sync(0xffffffffu, redo);
+            float f = 1.0f;
+            if (any_redo) {
+                // the offset is too low for this tile (or a score is not finite):
+                // move it to the row's max and redo P_j; O is rescaled below
+                const float hm = redo ? row_max<64>(x) * scale : -INFINITY;
+                xch[s * 256 + mine] = hm;
+                named_bar_sync(pair_bar, 64);
+                if (redo) {
+                    const float mn = fmaxf(m, fmaxf(hm, xch[s * 256 + theirs]));
+                    f = ex2(m - mn);
+                    m = mn;
+                }
+                lt = exp_scores<64>(x, scale, -m, pk);
+            }
+            if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
+            l = fmaf(l, f, lt);
+            // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE], (j - 1) & 1, abort_word, a.flags, a.wait_ns));
+                if (!ok) continue;
                 tc_fence_after();
-                const float inv_l = 1.0f / l;
-                const float inv_out = a.mix ? inv_l * a.mix[bh * 2] : inv_l;
-                const uint32_t qbuf = (t == 0 ? QA : QB);
+            }
+            if (any_redo && j > 0) {
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    float o[32], e[32];
-                    tmem_ld32(tO + c, o);
-                    if (inter) tmem_ld32(tS + c, e);
+                for (int c = 0; c < 64; c += 32) {
+                    float o[32];
+                    tmem_ld32(tO + lrow + cs + c, o);
                     tmem_ld_wait();
-                    if (!inter) {
-                        if (a.oi_ext && tok < T) {
-                            // token-level access: the read comes from the token-level kernels
-                            const float4* src = reinterpret_cast<const float4*>(
-                                a.oi_ext + (((size_t)b * T + tok) * a.H + h) * 128 + c);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 v = src[q];
-                                e[4 * q] = v.x;
-                                e[4 * q + 1] = v.y;
-                                e[4 * q + 2] = v.z;
-                                e[4 * q + 3] = v.w;
-                            }
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) e[q] = 0.f;
-                        }
-                    }
-                    if (a.out) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 w;
-                            w.x = pack_bf16(fmaf(o[8 * q + 0], inv_out, e[8 * q + 0]), fmaf(o[8 * q + 1], inv_out, e[8 * q + 1]));
-                            w.y = pack_bf16(fmaf(o[8 * q + 2], inv_out, e[8 * q + 2]), fmaf(o[8 * q + 3], inv_out, e[8 * q + 3]));
-                            w.z = pack_bf16(fmaf(o[8 * q + 4], inv_out, e[8 * q + 4]), fmaf(o[8 * q + 5], inv_out, e[8 * q + 5]));
-                            w.w = pack_bf16(fmaf(o[8 * q + 6], inv_out, e[8 * q + 6]), fmaf(o[8 * q + 7], inv_out, e[8 * q + 7]));
-                            // column chunk (c + 8q) / 8 of the row, in box c / 64
-                            const int chunk = (c % 64) / 8 + q;
-                            *reinterpret_cast<uint4*>(smem + qbuf + (c / 64) * kHalf + sw128_offset(r, chunk)) = w;
-                        }
-                    }
-                    if (a.out_intra && tok < T) {
-                        const size_t row = (((size_t)b * T + tok) * a.H + h) * 128 + c;
-                        float4* di = reinterpret_cast<float4*>(a.out_intra + row);
-                        float4* de = reinterpret_cast<float4*>(a.out_inter + row);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
-                                                o[4 * q + 3] * inv_l);
-                            de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
-                        }
-                    }
+                    for (int q = 0; q < 32; ++q) o[q] *= f;
+                    tmem_st32(tO + lrow + cs + c, o);
                 }
-                if (a.out) fence_async_smem();
             }
-            // the four warps of the tile meet here (no early exit); the tile is
-            // stored only if all of them wrote their rows
-            const bool all_ok = named_bar_and(1 + t, 128, e_ok);
-            if (a.out && all_ok && (threadIdx.x & 127) == 0) {
-                const uint32_t qbuf = (t == 0 ? QA : QB);
-                // rows past T are clipped by the tensor map
-                tma_store_3d(&tm_o, sb + qbuf, xh, q0, b);
-                tma_store_3d(&tm_o, sb + qbuf + kHalf, xh + 64, q0, b);
-                bulk_commit_group();
-                bulk_wait_read_all();
+            tmem_st32u(tP + lrow + hf * 32, pk);
+            // this half of S_{j+1} into registers while P_j is being stored
+            if (j + 1 < n) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + (s ^ 1)], ((j + 1) >> 1) & 1, abort_word,
+                                                       a.flags, a.wait_ns));
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t src = tS0 + (s ^ 1) * 128 + lrow + cs;
+                    tmem_ld32(src, x);
+                    tmem_ld32(src + 32, x + 32);
+                }
             }
+            tmem_st_wait();
+            tc_fence_before();
+            if (ok) mbar_arrive(&bars[B_PFULL]);
+        }
+        // epilogue: out = O / l + O_inter for this half of the row
+        if (ok) tmem_ld_wait();
+        bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags, a.wait_ns);
+        e_ok = __all_sync(0xffffffffu, e_ok && (!inter || mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags, a.wait_ns)));
+        // row sum over the two halves (slot parity n&1: its last readers passed
+        // the pair barrier of tile n-1)
+        xch[(n & 1) * 256 + mine] = l;
+        xfl[(n & 1) * 256 + mine] = e_ok ? 1 : 0;
+        named_bar_sync(pair_bar, 64);
+        const bool both = __all_sync(0xffffffffu, e_ok && xfl[(n & 1) * 256 + theirs] != 0);
+        if (both) {
+            tc_fence_after();
+            const float inv_l = 1.0f / (l + xch[(n & 1) * 256 + theirs]);  // commutative: the same in both halves
+            // out = a O_intra + O_inter (the inter gain c is folded into W); a = 1 without a mix
+            const float inv_out = a.mix ? inv_l * a.mix[bh * 2] : inv_l;
+            const int t = q0 + r;
+            const size_t row = (((size_t)b * T + t) * a.H + h) * 128 + cs;
+            float o[64], e[64];
+            tmem_ld32(tO + lrow + cs, o);
+            tmem_ld32(tO + lrow + cs + 32, o + 32);
+            if (inter) {
+                tmem_ld32(tOI + lrow + cs, e);
+                tmem_ld32(tOI + lrow + cs + 32, e + 32);
+            } else if (a.oi_ext && t < T) {
+                // token-level access: the read comes from the token-level kernels
+                const float4* src = reinterpret_cast<const float4*>(a.oi_ext + row);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float4 v = src[q];
+                    e[4 * q] = v.x;
+                    e[4 * q + 1] = v.y;
+                    e[4 * q + 2] = v.z;
+                    e[4 * q + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 64; ++q) e[q] = 0.f;
+            }
+            tmem_ld_wait();
+            if (a.out) {
+                // bf16 half-row into box hf of the (free) Q buffer, 128B-swizzled
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16(o[8 * q + 0] * inv_out + e[8 * q + 0], o[8 * q + 1] * inv_out + e[8 * q + 1]);
+                    w.y = pack_bf16(o[8 * q + 2] * inv_out + e[8 * q + 2], o[8 * q + 3] * inv_out + e[8 * q + 3]);
+                    w.z = pack_bf16(o[8 * q + 4] * inv_out + e[8 * q + 4], o[8 * q + 5] * inv_out + e[8 * q + 5]);
+                    w.w = pack_bf16(o[8 * q + 6] * inv_out + e[8 * q + 6], o[8 * q + 7] * inv_out + e[8 * q + 7]);
+                    *reinterpret_cast<uint4*>(smem + Q + hf * kHalf + sw128_offset(r, q)) = w;
+                }
+                fence_async_smem();
+            }
+            if (a.out_intra && t < T) {
+                float4* di = reinterpret_cast<float4*>(a.out_intra + row);
+                float4* de = reinterpret_cast<float4*>(a.out_inter + row);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    di[q] = make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l,
+                                        o[4 * q + 3] * inv_l);
+                    de[q] = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
+                }
+            }
+        }
+        // every softmax warp reaches this barrier (no early exit); the tile is
+        // stored only if all eight wrote their half-rows
+        if (!both && lane == 0) *epi_bad = 1;
+        named_bar_sync(5, kSoftmaxThreads);
+        if (a.out && threadIdx.x == 0 && *epi_bad == 0) {
+            // rows past T are clipped by the tensor map
+            tma_store_3d(&tm_o, sb + Q, h * 128, q0, b);
+            tma_store_3d(&tm_o, sb + Q + kHalf, h * 128 + 64, q0, b);
+            bulk_commit_group();
+            bulk_wait_read_all();
         }
     }
     tc_fence_before();
@@ -456,6 +487,7 @@ __global__ void __launch_bounds__(pp::kThreads, 1)
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
+
 
 }  // namespace tc
 }  // namespace hyb

@@ -183,23 +183,29 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
         for (int i = lane; i < D; i += 32) Kp[t * D + i] *= inv;
     }
     __syncthreads();
-    // L (strictly lower, decayed, beta-scaled k'.k') and the masked decayed q'.k'
-    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+    // L (strictly lower, decayed, beta-scaled k'.k') and the masked decayed q'.k':
+    // a warp per pair (t, s), its lanes over the feature index
+    for (int e = warp; e < kChunk * kChunk; e += kThreads / 32) {
         const int t = e / kChunk, s = e % kChunk;
         float l = 0.f, qk = 0.f;
         if (s < t) {
             float dk = 0.f, dq = 0.f;
-            for (int i = 0; i < D; ++i) {
+#pragma unroll
+            for (int i = lane; i < D; i += 32) {
                 const float ks = Kp[s * D + i];
                 dk = fmaf(Kp[t * D + i], ks, dk);
                 dq = fmaf(Qp[t * D + i], ks, dq);
             }
+            dk = warp_sum(dk);
+            dq = warp_sum(dq);
             const float dd = expf(fminf(lam[t - 1] - lam[s], 0.f));
             l = bet[t] * dd * dk;
             qk = dd * dq;
         }
-        Ls[e] = l;
-        rec[R::QK + e] = qk;
+        if (lane == 0) {
+            Ls[e] = l;
+            rec[R::QK + e] = qk;
+        }
     }
     // right-hand sides [beta V' | beta gprev K'] and the forward substitution,
     // one column per thread
@@ -210,9 +216,17 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
     __syncthreads();
     for (int j = tid; j < 2 * D; j += kThreads) {
         for (int t = 1; t < kChunk; ++t) {
-            float x = Sol[t * 2 * D + j];
-            for (int s = 0; s < t; ++s) x = fmaf(-Ls[t * kChunk + s], Sol[s * 2 * D + j], x);
-            Sol[t * 2 * D + j] = x;
+            // four independent partial sums (the chain over s is the latency)
+            float x0 = Sol[t * 2 * D + j], x1 = 0.f, x2 = 0.f, x3 = 0.f;
+            int s = 0;
+            for (; s + 4 <= t; s += 4) {
+                x0 = fmaf(-Ls[t * kChunk + s], Sol[s * 2 * D + j], x0);
+                x1 = fmaf(-Ls[t * kChunk + s + 1], Sol[(s + 1) * 2 * D + j], x1);
+                x2 = fmaf(-Ls[t * kChunk + s + 2], Sol[(s + 2) * 2 * D + j], x2);
+                x3 = fmaf(-Ls[t * kChunk + s + 3], Sol[(s + 3) * 2 * D + j], x3);
+            }
+            for (; s < t; ++s) x0 = fmaf(-Ls[t * kChunk + s], Sol[s * 2 * D + j], x0);
+            Sol[t * 2 * D + j] = (x0 + x1) + (x2 + x3);
         }
     }
     __syncthreads();
@@ -266,15 +280,16 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
 // every chunk's start state is saved for the reads, S_N goes to the state.
 template <int D>
 struct ChainSmem {
-    static constexpr size_t bytes = sizeof(float) * ((size_t)D * D + (size_t)D * kBand);
+    // M with rows padded to D + 1 floats (thread i reads row i: no bank conflicts)
+    static constexpr size_t bytes = sizeof(float) * ((size_t)D * (D + 1) + (size_t)D * kBand);
 };
 
 template <int D>
 __global__ void __launch_bounds__(D) chunk_chain_kernel(LayerArgs a, float* __restrict__ rec_base) {
     using R = Rec<D>;
     extern __shared__ __align__(16) float csm[];
-    float* Ms = csm;                                   // [D][D]
-    float (*Ss)[kBand] = reinterpret_cast<float (*)[kBand]>(csm + (size_t)D * D);
+    float* Ms = csm;                                   // [D][D + 1]
+    float (*Ss)[kBand] = reinterpret_cast<float (*)[kBand]>(csm + (size_t)D * (D + 1));
     const int band = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j0 = band * kBand;
     const int i = threadIdx.x;  // row of S
@@ -292,13 +307,21 @@ __global__ void __launch_bounds__(D) chunk_chain_kernel(LayerArgs a, float* __re
             Ss[i][j] = s[j];
         }
         const float4* M4 = reinterpret_cast<const float4*>(rec + R::M);
-        for (int e = i; e < D * D / 4; e += D) reinterpret_cast<float4*>(Ms)[e] = M4[e];
+        for (int e = i; e < D * D / 4; e += D) {
+            const float4 v = M4[e];
+            const int r = (4 * e) / D, cc = (4 * e) % D;
+            float* dst = Ms + r * (D + 1) + cc;
+            dst[0] = v.x;
+            dst[1] = v.y;
+            dst[2] = v.z;
+            dst[3] = v.w;
+        }
         __syncthreads();
         float acc[kBand];
 #pragma unroll
         for (int j = 0; j < kBand; ++j) acc[j] = rec[R::N + (size_t)i * D + j0 + j];
         for (int k = 0; k < D; ++k) {
-            const float mik = Ms[i * D + k];
+            const float mik = Ms[i * (D + 1) + k];
 #pragma unroll
             for (int j = 0; j < kBand; ++j) acc[j] = fmaf(mik, Ss[k][j], acc[j]);
         }
