@@ -313,8 +313,15 @@ def run_cuda(args):
     # the streaming step: 4 query-only passes and a clean pass of one frame)
     cleans = [int(c) for _ in range(w.frames) for c in w.passes]
     host = [W.pass_inputs(w, n, p) for n in range(w.frames) for p in range(len(w.passes))]
-    frames = [[t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)] for x in host]
-    outs = [torch.empty_like(f[0]) for f in frames]
+    # inputs and outputs of all passes stacked ([pass][B][T][H][d], [pass][B][H][T]);
+    # the per-pass calls use views of the same memory
+    stk = [torch.stack([getattr(x, f) for x in host]).to(dev).contiguous()
+           for f in ("q", "k", "v", "gate_logits", "beta_logits")]
+    frames = [[t[n] for t in stk] for n in range(len(host))]
+    out_stk = torch.empty_like(stk[0])
+    outs = [out_stk[n] for n in range(len(host))]
+    # one call for the whole stream of clean passes (hyb_attn_forward_frames)
+    frames_api = all(w.passes)
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
     wsb = layer.workspace.numel()
@@ -337,12 +344,26 @@ def run_cuda(args):
         torch.cuda.synchronize(dev)
         state0.copy_(layer.state)
 
-    def step():
+    def step_loop():
         layer.state.copy_(state0)
         for c in calls:
             st = fwd(dref, *c)
             if st != G.HYB_OK:
                 raise G.HybAttnError(st, "hyb_attn_forward")
+
+    if frames_api:
+        nf = len(host)
+        fws = torch.zeros(G.hyb_attn_frames_workspace_bytes(desc, nf), dtype=torch.uint8, device=dev)
+        fcall = [dref, nf, stk[0].data_ptr(), stk[1].data_ptr(), stk[2].data_ptr(), *phis, stk[3].data_ptr(),
+                 stk[4].data_ptr(), state_ptr, out_stk.data_ptr(), fws.data_ptr(), fws.numel(), sptr]
+
+        def step():
+            layer.state.copy_(state0)
+            st = G.lib.hyb_attn_forward_frames(*fcall)
+            if st != G.HYB_OK:
+                raise G.HybAttnError(st, "hyb_attn_forward_frames")
+    else:
+        step = step_loop
 
     if args.profile_run:
         # kernel order per frame: prep, intra_frame_attention, delta_update
@@ -354,6 +375,7 @@ def run_cuda(args):
 
     for _ in range(max(3, args.warmup)):
         step()
+        step_loop()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -369,19 +391,33 @@ def run_cuda(args):
         stop.record(stream)
         torch.cuda.synchronize(dev)
     ms = max_over_ranks(start.elapsed_time(stop), dev)
-    # timed region B: the same steps with the library's timing hook, which brackets
-    # every kernel with events on the library's stream (per-kernel durations)
+    # the same steps as one hyb_attn_forward call per pass (autoregressive use:
+    # the next frame's inputs exist only after this frame)
+    ms_loop = ms
+    if frames_api:
+        if world > 1:
+            dist.barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            step_loop()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_loop = max_over_ranks(start.elapsed_time(stop), dev)
+    # timed region B: the per-pass calls with the library's timing hook, which
+    # brackets every kernel with events on the library's stream (per-kernel durations)
     n_launch_cap = args.steps * w.frames * len(w.passes) * G.HYB_NUM_KERNELS + 16
     assert G.hyb_attn_timing_begin(n_launch_cap) == G.HYB_OK
     start.record(stream)
     for _ in range(args.steps):
-        step()
+        step_loop()
     stop.record(stream)
     torch.cuda.synchronize(dev)
     ms_hooked = start.elapsed_time(stop)
     st, per_kernel, dropped = G.hyb_attn_timing_end()
     assert st == G.HYB_OK and dropped == 0, (st, dropped)
     status = layer.device_status()
+    if frames_api and status == G.HYB_OK:
+        status = G.hyb_attn_get_device_status(fws)
 
     tokens_per_step = w.B * w.T * w.frames
     value = job_throughput(tokens_per_step, args.steps, world, ms)
@@ -429,6 +465,17 @@ def run_cuda(args):
 
     def e2e_step():
         layer.state.copy_(state0)
+        if frames_api:
+            # every frame's inputs in, one call, every frame's output back
+            for f, hf in zip(frames, pin):
+                for dst, src_ in zip(f, hf):
+                    dst.copy_(src_, non_blocking=True)
+            st = G.lib.hyb_attn_forward_frames(*fcall)
+            if st != G.HYB_OK:
+                raise G.HybAttnError(st, "hyb_attn_forward_frames")
+            for o, ho in zip(outs, hout):
+                ho.copy_(o, non_blocking=True)
+            return
         for f, hf, c, o, ho in zip(frames, pin, calls, outs, hout):
             for dst, src_ in zip(f, hf):
                 dst.copy_(src_, non_blocking=True)
@@ -477,6 +524,11 @@ def run_cuda(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "api": ("hyb_attn_forward_frames (one call per 21-frame forward; bit-identical to one "
+                "hyb_attn_forward call per frame)") if frames_api else "hyb_attn_forward (one call per pass)",
+        "per_frame_calls": {"value": job_throughput(tokens_per_step, args.steps, world, ms_loop), "unit": UNIT,
+                            "us_per_frame": 1e3 * ms_loop / args.steps / w.frames,
+                            "api": "hyb_attn_forward, one call per pass (the autoregressive pattern)"},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "device_status": G.hyb_attn_status_string(status),

@@ -35,6 +35,8 @@ from ._binding import (  # noqa: F401
     HybridAttention,
     TokenLevelAttention,
     hyb_attn_forward_token_level,
+    hyb_attn_forward_frames,
+    hyb_attn_frames_workspace_bytes,
     hyb_attn_token_level_workspace_bytes,
     KVCacheAttention,
     HybAttnTiming,

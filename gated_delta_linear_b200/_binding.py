@@ -62,6 +62,10 @@ def _load():
     L.hyb_attn_forward_noalloc.restype = i
     L.hyb_attn_forward_mixed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.hyb_attn_forward_mixed.restype = i
+    L.hyb_attn_frames_workspace_bytes.argtypes = [dp, i]
+    L.hyb_attn_frames_workspace_bytes.restype = sz
+    L.hyb_attn_forward_frames.argtypes = [dp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.hyb_attn_forward_frames.restype = i
     L.hyb_attn_token_level_workspace_bytes.argtypes = [dp]
     L.hyb_attn_token_level_workspace_bytes.restype = sz
     L.hyb_attn_forward_token_level.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
@@ -144,6 +148,19 @@ def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, be
                                         _ptr(phi_q), _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits),
                                         _ptr(beta_logits), _ptr(state), int(clean_pass), _ptr(out),
                                         _stream(stream))
+
+
+def hyb_attn_frames_workspace_bytes(desc: HybAttnDesc, n_frames: int) -> int:
+    return lib.hyb_attn_frames_workspace_bytes(ctypes.byref(desc), int(n_frames))
+
+
+def hyb_attn_forward_frames(desc, n_frames, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                            out, workspace, workspace_bytes=None, stream=None) -> int:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_attn_forward_frames(ctypes.byref(desc), int(n_frames), _ptr(q), _ptr(k), _ptr(v), _ptr(phi_q),
+                                       _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits), _ptr(beta_logits),
+                                       _ptr(state), _ptr(out), _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def hyb_attn_token_level_workspace_bytes(desc: HybAttnDesc) -> int:

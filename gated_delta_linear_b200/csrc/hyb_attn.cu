@@ -192,7 +192,7 @@ struct MapKey {
     }
 };
 struct MapCache {
-    static constexpr int kEntries = 32;
+    static constexpr int kEntries = 128;
     MapKey key[kEntries];
     CUtensorMap map[kEntries];
     int used = 0, next = 0;
@@ -226,74 +226,106 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
     return true;
 }
 
-cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
-    static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
-    constexpr int D = 128;
-    cudaError_t e;
-    if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
-    if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
-    const uint64_t row_bytes = (uint64_t)a.H * D * 2;
-    const uint64_t bh = (uint64_t)a.B * a.H;
+// The three kernels of one bf16 pass: tensor maps encoded once, each kernel
+// launchable on a given stream, as a programmatic dependent of the previous
+// kernel of that stream or not.
+struct TcPass {
+    LayerArgs a;
     CUtensorMap tq, tk, tv, tw, tphik, tphiq, tout;
-    if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
-        (a.out && !map3d(&tout, a.out, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T)) ||
-        !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
-        !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
-        !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
-        !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2) ||
-        !map3d(&tphiq, a.phi_q, D, D, a.H, D * 2, D * D * 2))
-        return cudaErrorInvalidValue;
-    if (!a.out) tout = tq;  // not read: the attention kernel stores no bf16 output
-    // Kernels of a pass are chained by programmatic dependent launch: prep waits
-    // for the previous kernel of the stream before it reads the state, then lets
-    // the attention kernel start, which reads prep's W only at its end.
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t pcfg = {};
-    pcfg.gridDim = dim3(1, a.H, a.B);
-    pcfg.blockDim = dim3(tc::prep::kThreads, 1, 1);
-    pcfg.dynamicSmemBytes = tc::prep::SMEM;
-    pcfg.stream = st;
-    pcfg.attrs = pdl;
-    pcfg.numAttrs = 1;
-    cudaError_t le = cudaSuccess;
-    e = timed(K_PREP, st, [&] { le = cudaLaunchKernelEx(&pcfg, tc::prep_tc_kernel, a, tphiq); });
-    if (e != cudaSuccess) return e;
-    if (le != cudaSuccess) return le;
-    cudaLaunchConfig_t acfg = {};
-    acfg.gridDim = dim3(attn_tiles(a.T), a.H, a.B);
-    acfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
-    acfg.dynamicSmemBytes = tc::attn::SMEM;
-    acfg.stream = st;
-    acfg.attrs = pdl;
-    acfg.numAttrs = 1;
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tw, tout); });
-    if (e != cudaSuccess) return e;
-    if (le != cudaSuccess) return le;
-    if (clean) {
+
+    cudaError_t init(const LayerArgs& args) {
+        static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
+        constexpr int D = 128;
+        a = args;
+        cudaError_t e;
+        if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
+        const uint64_t row_bytes = (uint64_t)a.H * D * 2;
+        const uint64_t bh = (uint64_t)a.B * a.H;
+        if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            (a.out && !map3d(&tout, a.out, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T)) ||
+            !map3d(&tk, a.k, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            !map3d(&tv, a.v, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
+            !map3d(&tw, a.WT_hi, D, D, 2 * bh, D * 2, D * D * 2) ||
+            !map3d(&tphik, a.phi_k, D, D, a.H, D * 2, D * D * 2) ||
+            !map3d(&tphiq, a.phi_q, D, D, a.H, D * 2, D * D * 2))
+            return cudaErrorInvalidValue;
+        if (!a.out) tout = tq;  // not read: the attention kernel stores no bf16 output
+        return cudaSuccess;
+    }
+
+    static void pdl_attr(cudaLaunchAttribute* at) {
+        at->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at->val.programmaticStreamSerializationAllowed = 1;
+    }
+
+    cudaError_t prep(cudaStream_t st, bool pdl) {
+        cudaLaunchAttribute at[1];
+        pdl_attr(&at[0]);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, a.H, a.B);
+        cfg.blockDim = dim3(tc::prep::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = tc::prep::SMEM;
+        cfg.stream = st;
+        cfg.attrs = at;
+        cfg.numAttrs = pdl ? 1 : 0;
+        cudaError_t le = cudaSuccess;
+        cudaError_t e = timed(K_PREP, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::prep_tc_kernel, a, tphiq); });
+        return e != cudaSuccess ? e : le;
+    }
+
+    cudaError_t attn(cudaStream_t st, bool pdl) {
+        cudaLaunchAttribute at[1];
+        pdl_attr(&at[0]);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(attn_tiles(a.T), a.H, a.B);
+        cfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = tc::attn::SMEM;
+        cfg.stream = st;
+        cfg.attrs = at;
+        cfg.numAttrs = pdl ? 1 : 0;
+        cudaError_t le = cudaSuccess;
+        cudaError_t e = timed(K_ATTN, st, [&] {
+            le = cudaLaunchKernelEx(&cfg, tc::attention_kernel, a, tq, tk, tv, tw, tout);
+        });
+        return e != cudaSuccess ? e : le;
+    }
+
+    cudaError_t update(cudaStream_t st, bool pdl) {
         // one cluster of nsplit CTAs per (b, h)
+        cudaLaunchAttribute at[2];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = a.nsplit;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        pdl_attr(&at[1]);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(a.nsplit, a.H, a.B);
         cfg.blockDim = dim3(tc::upd::kThreads, 1, 1);
         cfg.dynamicSmemBytes = tc::upd::SMEM;
         cfg.stream = st;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = a.nsplit;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        // programmatic dependent of the attention kernel: may run on the SMs its
-        // last wave leaves idle (it reads only inputs and prep's outputs)
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 2;
-        e = timed(K_UPDATE, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik); });
-        if (e != cudaSuccess) return e;
-        if (le != cudaSuccess) return le;
+        cfg.attrs = at;
+        cfg.numAttrs = pdl ? 2 : 1;
+        cudaError_t le = cudaSuccess;
+        cudaError_t e = timed(K_UPDATE, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik); });
+        return e != cudaSuccess ? e : le;
     }
+};
+
+cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
+    TcPass tp;
+    cudaError_t e = tp.init(a);
+    if (e != cudaSuccess) return e;
+    // Kernels of a pass are chained by programmatic dependent launch: prep waits
+    // for the previous kernel of the stream, then lets the attention kernel start
+    // (which reads prep's W only at its end, after waiting for prep) and reads the
+    // state; the delta update starts beside the attention kernel (on the SMs its
+    // last wave leaves idle) and writes the state only after the attention grid,
+    // and so prep, has completed.
+    if ((e = tp.prep(st, true)) != cudaSuccess) return e;
+    if ((e = tp.attn(st, true)) != cudaSuccess) return e;
+    if (clean && (e = tp.update(st, true)) != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -443,6 +475,65 @@ hyb_status launch_pass(const LayerArgs& a, const Plan& p, int clean_pass, void* 
     return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
+// ---- several frames in one call ---------------------------------------------------
+// Per device: a high-priority stream for the state chain (prep, update of each
+// frame), a stream for the attention kernels, and events; created on the first
+// call on the device and kept.  The calls are not thread-safe.
+struct FrameRes {
+    bool ready = false;
+    cudaStream_t chain = nullptr, att = nullptr;
+    cudaEvent_t fork = nullptr, join_chain = nullptr, join_att = nullptr;
+    cudaEvent_t* w = nullptr;
+    int nw = 0;
+};
+FrameRes g_frames[kMaxDevices];
+constexpr int kMaxFrames = 4096;
+
+cudaError_t frame_resources(int n, FrameRes** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    FrameRes& r = g_frames[dev];
+    if (!r.ready) {
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&r.chain, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&r.att, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&r.join_chain, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&r.join_att, cudaEventDisableTiming)) != cudaSuccess) return e;
+        r.ready = true;
+    }
+    if (r.nw < n) {
+        cudaEvent_t* w = new (std::nothrow) cudaEvent_t[n];
+        if (!w) return cudaErrorMemoryAllocation;
+        int made = 0;
+        for (; made < n; ++made)
+            if ((e = cudaEventCreateWithFlags(&w[made], cudaEventDisableTiming)) != cudaSuccess) break;
+        if (made < n) {
+            for (int i = 0; i < made; ++i) cudaEventDestroy(w[i]);
+            delete[] w;
+            return e;
+        }
+        // events of earlier calls: the waits on them were enqueued by those calls
+        for (int i = 0; i < r.nw; ++i) cudaEventDestroy(r.w[i]);
+        delete[] r.w;
+        r.w = w;
+        r.nw = n;
+    }
+    *out = &r;
+    return cudaSuccess;
+}
+
+size_t frames_w_bytes(const hyb_attn_desc* d, const Plan& p) {
+    return (size_t)d->B * d->H * p.D * p.D * 2 * sizeof(__nv_bfloat16);
+}
+
+size_t frames_total(const hyb_attn_desc* d, const Plan& p, int n) {
+    return align_up(p.total, 256) + (p.bf16 ? (size_t)n * align_up(frames_w_bytes(d, p), 256) : 0);
+}
+
 hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
                         const void* phi_q, const void* phi_k, const void* phi_v,
                         const float* gate_logits, const float* beta_logits, float* state,
@@ -576,6 +667,87 @@ hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc, const void* q, cons
     if (!mix || !out) return HYB_ERR_INVALID;
     return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out,
                         nullptr, nullptr, workspace, workspace_bytes, stream, mix);
+}
+
+size_t hyb_attn_frames_workspace_bytes(const hyb_attn_desc* desc, int n_frames) {
+    Plan p;
+    if (n_frames < 1 || n_frames > kMaxFrames || make_plan(desc, &p) != HYB_OK) return 0;
+    return frames_total(desc, p, n_frames);
+}
+
+hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, const void* q, const void* k,
+                                   const void* v, const void* phi_q, const void* phi_k, const void* phi_v,
+                                   const float* gate_logits, const float* beta_logits, float* state, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    Plan p;
+    hyb_status s = make_plan(desc, &p);
+    if (s != HYB_OK) return s;
+    if (n_frames < 1 || n_frames > kMaxFrames) return HYB_ERR_INVALID;
+    if (!q || !k || !v || !out || !gate_logits || !beta_logits) return HYB_ERR_INVALID;
+    if (!workspace || workspace_bytes < frames_total(desc, p, n_frames)) return HYB_ERR_WORKSPACE;
+    const size_t esz = p.bf16 ? 2 : 4;
+    const size_t fe = (size_t)desc->B * desc->T * desc->H * p.D * esz;  // bytes of q (k, v, out) per frame
+    const size_t fg = (size_t)desc->B * desc->H * desc->T;              // gate logits per frame
+    LayerArgs* args = new (std::nothrow) LayerArgs[n_frames];
+    if (!args) return HYB_ERR_INVALID;
+    // every frame's arguments are checked before anything is enqueued
+    for (int n = 0; n < n_frames && s == HYB_OK; ++n)
+        s = pass_args(desc, (const char*)q + n * fe, (const char*)k + n * fe, (const char*)v + n * fe, phi_q, phi_k,
+                      phi_v, gate_logits + n * fg, beta_logits + n * fg, state, 1, (char*)out + n * fe, nullptr,
+                      nullptr, workspace, workspace_bytes, nullptr, &args[n], &p);
+    if (s != HYB_OK) {
+        delete[] args;
+        return s;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (!p.bf16) {
+        // fp32 path: the frames one after another on the caller's stream
+        for (int n = 0; n < n_frames && e == cudaSuccess; ++n) e = launch_simt<32, float>(args[n], 1, st);
+        delete[] args;
+        return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+    }
+    // bf16: the state chain (W_N = phi_q^T S_{N-1}, then S_N) on one stream, the
+    // attention kernels on another; attention of frame N waits only for W_N, so
+    // the attention kernels of consecutive frames share the SMs instead of each
+    // ending on a partial wave.  Each frame's W has its own slot.
+    FrameRes* r = nullptr;
+    if ((e = frame_resources(n_frames, &r)) != cudaSuccess) {
+        delete[] args;
+        return HYB_ERR_CUDA;
+    }
+    const size_t wslot = align_up(frames_w_bytes(desc, p), 256);
+    char* slots = (char*)workspace + align_up(p.total, 256);
+    const size_t hh = (size_t)desc->B * desc->H * p.D * p.D;
+    TcPass* tp = new (std::nothrow) TcPass[n_frames];
+    if (!tp) {
+        delete[] args;
+        return HYB_ERR_INVALID;
+    }
+    for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
+        args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
+        args[n].WT_lo = args[n].WT_hi + hh;
+        e = tp[n].init(args[n]);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(r->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(r->chain, r->fork, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(r->att, r->fork, 0);
+    for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
+        if ((e = tp[n].prep(r->chain, false)) != cudaSuccess) break;
+        if ((e = cudaEventRecord(r->w[n], r->chain)) != cudaSuccess) break;
+        if ((e = tp[n].update(r->chain, false)) != cudaSuccess) break;
+        if ((e = cudaStreamWaitEvent(r->att, r->w[n], 0)) != cudaSuccess) break;
+        e = tp[n].attn(r->att, false);
+    }
+    // join: the caller's stream continues after every frame's kernels
+    if (e == cudaSuccess) e = cudaEventRecord(r->join_chain, r->chain);
+    if (e == cudaSuccess) e = cudaEventRecord(r->join_att, r->att);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, r->join_chain, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, r->join_att, 0);
+    delete[] tp;
+    delete[] args;
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
 size_t hyb_attn_token_level_workspace_bytes(const hyb_attn_desc* desc) {

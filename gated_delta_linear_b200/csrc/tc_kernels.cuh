@@ -466,6 +466,10 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         wsum[10] = t / (float)T;
     }
     cluster_sync();  // every CTA of the cluster has parked Delta_c and staged S_{N-1}
+    // S_N overwrites S_{N-1} in place: wait until the attention grid of this pass
+    // has completed.  It waited for the prep grid before loading W, so every read
+    // of S_{N-1} for this frame's output is done by then.
+    pdl_wait_primary();
 
     // ------------------------------------------------------------ reduce and apply this CTA's band
     // S_N[row] = alpha S_{N-1}[row] + sum_c Delta_c[row], ranks summed in order
@@ -512,9 +516,6 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     cluster_sync();  // no CTA leaves while another still reads its shared memory
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
-    // when launched as a programmatic dependent of the attention kernel, complete
-    // only after it: later work in the stream stays ordered after both
-    pdl_wait_primary();
 }
 
 // ============================================================== prep: W = phi_q^T S_{N-1}
@@ -563,8 +564,12 @@ __global__ void __launch_bounds__(prep::kThreads, 1)
     }
     if (warp == 0) tmem_alloc(tmem_slot, 128);
     // launched as a programmatic dependent: the previous kernel of the stream may
-    // write the state, so wait for it before reading S_{N-1}
+    // write the state, so wait for it before reading S_{N-1}; then let the
+    // attention kernel start (it needs W only at its end, after this grid has
+    // completed).  The delta update launched behind it writes the state only
+    // after the attention grid has completed, and so after every read below.
     pdl_wait_primary();
+    pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -574,10 +579,6 @@ __global__ void __launch_bounds__(prep::kThreads, 1)
         bulk_load(sb + SF, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_S]);
     }
     const bool s_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_S], 0, abort_word, a.flags, a.wait_ns));
-    // S_{N-1} is in shared memory: only now may the attention kernel start, and
-    // through it the delta update that overwrites the state in place
-    __syncthreads();
-    pdl_launch_dependents();
     const int half = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     if (s_ok) {

@@ -113,6 +113,35 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
                                      float* out_intra, float* out_inter,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* hyb_attn_forward_frames -- n_frames consecutive frames of one stream, each a
+ * clean pass (hyb_attn_forward with clean_pass = 1, frame after frame), in one
+ * call.  The results are bit-identical to that loop: the same kernels with the
+ * same arithmetic; only their scheduling differs.  Frame N's inter-frame read
+ * needs W_N = phi_q^T S_{N-1} only at the end of its attention kernel, and
+ * frame N's state update never waits for frame N's attention, so the call runs
+ * the short sequential chain (W_N, then S_N, frame after frame) on one internal
+ * stream and the attention kernels on another, each attention kernel waiting
+ * only for its own W_N: the attention kernels of consecutive frames share the
+ * SMs.  The internal streams (the chain's at the highest priority) and events
+ * are created on the first call on a device and kept; the call forks from and
+ * joins back to `stream`, so work enqueued on `stream` afterwards sees every
+ * output and the final state.  Not thread-safe.
+ *   q, k, v, out: [n_frames][B][T][H][d]; gate_logits, beta_logits:
+ *   [n_frames][B][H][T] fp32 (B*H*T a multiple of 4, so every frame's gate
+ *   pointer stays 16-byte aligned; HYB_ERR_ALIGN otherwise); state: S_{-1} on
+ *   entry (the state before the first frame), the state after the last frame
+ *   on return.  workspace: hyb_attn_frames_workspace_bytes(desc, n_frames)
+ *   bytes (it grows with n_frames: one W per frame), zero-filled once.
+ * HYB_ERR_INVALID if n_frames is outside [1, 4096]; otherwise the errors of
+ * hyb_attn_forward, checked for every frame before anything is enqueued. */
+size_t hyb_attn_frames_workspace_bytes(const hyb_attn_desc* desc, int n_frames);
+hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames,
+                                   const void* q, const void* k, const void* v,
+                                   const void* phi_q, const void* phi_k, const void* phi_v,
+                                   const float* gate_logits, const float* beta_logits,
+                                   float* state, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* hyb_attn_forward_mixed -- the same pass with a per-(batch, head) weighting of
  * the two branches: out = a * O_intra + c * O_inter, with (a, c) = mix[b][h]
  * ([B][H][2] fp32, device memory, 16-byte aligned).  It carries the branch
