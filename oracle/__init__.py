@@ -9,7 +9,9 @@ or helpers with ``gated_delta_linear_b200``, and neither side imports the other.
 Source: "Technical summary: Attend Locally, Remember Linearly (ARL2)"
 (gist.science/ar/paper/2605.16579), §2.1 "hybrid attention decomposition"
 and §2.2 "memory-state management"; §1 for the key/value-cache softmax
-baseline (``kvcache_attention``).
+baseline (``kvcache_attention``).  ``oracle.tra``: Token Radius Attention
+("Technical summary: Token Radius Attention", gist.science/ar/paper/2608.02504)
+on the intra-frame branch.
 """
 
 from .hybrid_layer import (  # noqa: F401
@@ -27,3 +29,4 @@ from .hybrid_layer import (  # noqa: F401
     mixed_output,
     token_level_head_pass,
 )
+from . import tra  # noqa: F401
