@@ -40,6 +40,8 @@ struct LayerArgs {
     __nv_bfloat16* WT_hi;      // bf16 [BH][D][D]: phi_q^T S, row-major, high part (tensor path)
     __nv_bfloat16* WT_lo;      // bf16 [BH][D][D]: low part
     float* S_prev;             // fp32 [BH][D][D]: copy of S_{N-1} (fp32 path, clean pass)
+    __nv_bfloat16* w_next;     // if set, the delta update also writes W of the next frame,
+                               // phi_q^T S_N, here (hi plane; lo plane BH D^2 further)
     float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
     int nsplit;
     int split_tokens;

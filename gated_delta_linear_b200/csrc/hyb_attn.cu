@@ -308,7 +308,9 @@ struct TcPass {
         cfg.attrs = at;
         cfg.numAttrs = pdl ? 2 : 1;
         cudaError_t le = cudaSuccess;
-        cudaError_t e = timed(K_UPDATE, st, [&] { le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik); });
+        cudaError_t e = timed(K_UPDATE, st, [&] {
+            le = cudaLaunchKernelEx(&cfg, tc::update_kernel, a, tk, tv, tphik, tphiq);
+        });
         return e != cudaSuccess ? e : le;
     }
 };
@@ -318,11 +320,11 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     cudaError_t e = tp.init(a);
     if (e != cudaSuccess) return e;
     // Kernels of a pass are chained by programmatic dependent launch: prep waits
-    // for the previous kernel of the stream, then lets the attention kernel start
-    // (which reads prep's W only at its end, after waiting for prep) and reads the
-    // state; the delta update starts beside the attention kernel (on the SMs its
-    // last wave leaves idle) and writes the state only after the attention grid,
-    // and so prep, has completed.
+    // for the previous kernel of the stream and stages the state, then lets the
+    // attention kernel start (which reads prep's W only at its end, after waiting
+    // for prep); the delta update starts once every attention CTA has started (on
+    // the SMs the last wave leaves idle), so after prep has read the state it
+    // overwrites, and completes only after the attention grid.
     if ((e = tp.prep(st, true)) != cudaSuccess) return e;
     if ((e = tp.attn(st, true)) != cudaSuccess) return e;
     if (clean && (e = tp.update(st, true)) != cudaSuccess) return e;
@@ -727,15 +729,19 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
         args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
         args[n].WT_lo = args[n].WT_hi + hh;
+        // the update of frame n also writes W of frame n + 1 (what prep would
+        // compute from S_n), so the chain is one kernel per frame
+        args[n].w_next = n + 1 < n_frames ? (__nv_bfloat16*)(slots + (n + 1) * wslot) : nullptr;
         e = tp[n].init(args[n]);
     }
     if (e == cudaSuccess) e = cudaEventRecord(r->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(r->chain, r->fork, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(r->att, r->fork, 0);
+    if (e == cudaSuccess) e = tp[0].prep(r->chain, false);
+    if (e == cudaSuccess) e = cudaEventRecord(r->w[0], r->chain);
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
-        if ((e = tp[n].prep(r->chain, false)) != cudaSuccess) break;
-        if ((e = cudaEventRecord(r->w[n], r->chain)) != cudaSuccess) break;
         if ((e = tp[n].update(r->chain, false)) != cudaSuccess) break;
+        if (n + 1 < n_frames && (e = cudaEventRecord(r->w[n + 1], r->chain)) != cudaSuccess) break;
         if ((e = cudaStreamWaitEvent(r->att, r->w[n], 0)) != cudaSuccess) break;
         e = tp[n].attn(r->att, false);
     }

@@ -89,7 +89,7 @@ constexpr int kNormThreads = 256;                         // warps 0-7
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
 enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_KTFULL1, B_KTREAD, B_KTREAD1, B_OPSFULL, B_OPSFREE,
-       B_PARK, B_DELTA, B_COUNT };
+       B_PARK, B_DELTA, B_WPHI, B_WMMA, B_COUNT };
 static_assert(RED + 128 * 128 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
 // byte offset of float4 chunk q (0..31) of row `row` in RED
 __device__ __forceinline__ uint32_t red_off(int row, int q) {
@@ -123,7 +123,8 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t local_addr, uint32_t ra
 
 __global__ void __launch_bounds__(upd::kThreads, 1)
     update_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_phik) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_phik,
+                  const __grid_constant__ CUtensorMap tm_phiq) {
     using namespace upd;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023u) {  // uniform over the grid: every CTA leaves
@@ -465,11 +466,15 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         for (int w = 0; w < kThreads / 32; ++w) t += wsum[w];
         wsum[10] = t / (float)T;
     }
+    if (a.w_next && threadIdx.x == kLoadWarp * 32) {
+        // the Delta products have completed: phi_q (for the next frame's W) into
+        // the phi_v tile, as an MN-major A operand
+        tma_prefetch_desc(&tm_phiq);
+        mbar_expect_tx(&bars[B_WPHI], kTileBytes);
+        tma_load_3d(sb + PHIV, &tm_phiq, &bars[B_WPHI], 0, 0, h);
+        tma_load_3d(sb + PHIV + kHalf, &tm_phiq, &bars[B_WPHI], 64, 0, h);
+    }
     cluster_sync();  // every CTA of the cluster has parked Delta_c and staged S_{N-1}
-    // S_N overwrites S_{N-1} in place: wait until the attention grid of this pass
-    // has completed.  It waited for the prep grid before loading W, so every read
-    // of S_{N-1} for this frame's output is done by then.
-    pdl_wait_primary();
 
     // ------------------------------------------------------------ reduce and apply this CTA's band
     // S_N[row] = alpha S_{N-1}[row] + sum_c Delta_c[row], ranks summed in order
@@ -515,7 +520,92 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     }
     cluster_sync();  // no CTA leaves while another still reads its shared memory
     tc_fence_after();
+    if (a.w_next) {
+        // W_{N+1} = phi_q^T S_N for the next frame of a multi-frame call, with the
+        // prep kernel's operands and instruction sequence (so the same bits); every
+        // CTA of the cluster computes all of W and writes the rows of its band.  The
+        // cluster barrier above (release / acquire) makes every band of S_N visible.
+        const int half = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        if (warp < 8) {
+            const float4* Sg = reinterpret_cast<const float4*>(a.state + (size_t)bh * 128 * 128 + row * 128 + half * 64);
+            float4 sv[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sv[k] = __ldcg(Sg + k);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float4 v = sv[k];
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+                const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+                const uint2 hi = make_uint2(*reinterpret_cast<const uint32_t*>(&h01),
+                                            *reinterpret_cast<const uint32_t*>(&h23));
+                const uint2 lo = make_uint2(pack_bf16(v.x - __low2float(h01), v.y - __high2float(h01)),
+                                            pack_bf16(v.z - __low2float(h23), v.w - __high2float(h23)));
+                const uint32_t off = half * kHalf + sw128_offset(row, k >> 1) + (k & 1) * 8;
+                *reinterpret_cast<uint2*>(smem + SH + off) = hi;
+                *reinterpret_cast<uint2*>(smem + SL + off) = lo;
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (threadIdx.x == kMmaWarp * 32) {
+            if (park_ok && mbar_wait(&bars[B_WPHI], 0, abort_word, a.flags)) {
+                constexpr uint32_t ID_MNMN = idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tD, mnmajor_desc(sb + PHIV, kk), mnmajor_desc(sb + SH, kk), ID_MNMN, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tD, mnmajor_desc(sb + PHIV, kk), mnmajor_desc(sb + SL, kk), ID_MNMN, 1);
+            }
+            mma_commit(&bars[B_WMMA]);
+        }
+        if (warp < 8) {
+            const bool w_ok =
+                __all_sync(0xffffffffu, park_ok && mbar_wait(&bars[B_WMMA], 0, abort_word, a.flags));
+            const int band = (128 + C - 1) / C;
+            const int r0 = min(128, split * band), r1 = min(128, r0 + band);
+            if (w_ok) {
+                tc_fence_after();
+                const uint32_t lrow = (uint32_t)((warp & 3) * 32) << 16;
+                const size_t base = ((size_t)bh * 128 + row) * 128 + half * 64;
+                __nv_bfloat16* wlo = a.w_next + (size_t)a.B * a.H * 128 * 128;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    float x[32];
+                    tmem_ld32(tD + lrow + half * 64 + c * 32, x);
+                    tmem_ld_wait();
+                    if (row >= r0 && row < r1) {
+                        uint32_t hi[16], lo[16];
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const float w0 = x[2 * q] * 1.0f, w1 = x[2 * q + 1] * 1.0f;
+                            const __nv_bfloat162 hv = __floats2bfloat162_rn(w0, w1);
+                            hi[q] = *reinterpret_cast<const uint32_t*>(&hv);
+                            lo[q] = pack_bf16(w0 - __low2float(hv), w1 - __high2float(hv));
+                        }
+                        uint4* dh = reinterpret_cast<uint4*>(a.w_next + base + c * 32);
+                        uint4* dl = reinterpret_cast<uint4*>(wlo + base + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            dh[q] = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+                            dl[q] = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+    // when launched as a programmatic dependent of the attention kernel, complete
+    // only after it: later work in the stream (the next prep, which rewrites the
+    // W the attention kernel reads) stays ordered after both
+    pdl_wait_primary();
 }
 
 // ============================================================== prep: W = phi_q^T S_{N-1}
@@ -564,12 +654,8 @@ __global__ void __launch_bounds__(prep::kThreads, 1)
     }
     if (warp == 0) tmem_alloc(tmem_slot, 128);
     // launched as a programmatic dependent: the previous kernel of the stream may
-    // write the state, so wait for it before reading S_{N-1}; then let the
-    // attention kernel start (it needs W only at its end, after this grid has
-    // completed).  The delta update launched behind it writes the state only
-    // after the attention grid has completed, and so after every read below.
+    // write the state, so wait for it before reading S_{N-1}
     pdl_wait_primary();
-    pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -579,6 +665,11 @@ __global__ void __launch_bounds__(prep::kThreads, 1)
         bulk_load(sb + SF, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_S]);
     }
     const bool s_ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_S], 0, abort_word, a.flags, a.wait_ns));
+    // S_{N-1} is in shared memory: only now may the attention kernel start, and
+    // through it the delta update that overwrites the state in place (it is
+    // launched once every attention CTA has started)
+    __syncthreads();
+    pdl_launch_dependents();
     const int half = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     if (s_ok) {

@@ -52,7 +52,7 @@ struct Rec {
     static constexpr size_t U0 = Wm + (size_t)kChunk * D;         // [C][D] U0
     static constexpr size_t QK = U0 + (size_t)kChunk * D;         // [C][C] masked, decayed q'.k'
     static constexpr size_t GP = QK + (size_t)kChunk * kChunk;    // [C] gprev
-    static constexpr size_t M = GP + kChunk;                      // [D][D]
+    static constexpr size_t M = GP + kChunk;                      // [D][D] M^T (M[i][j] at j * D + i)
     static constexpr size_t N = M + (size_t)D * D;                // [D][D]
     static constexpr size_t S0 = N + (size_t)D * D;               // [D][D] the chunk's start state
     static constexpr size_t floats = (S0 + (size_t)D * D + 63) / 64 * 64;
@@ -63,7 +63,7 @@ struct PrepSmem {
     // phase 1: X [C][D+1] and phi^T [D][D]; K', V', Q' [C][D]; gates
     // phase 2 (reuses X / phi^T): L [C][C], [U0 | W] [C][2D]
     static constexpr size_t xs = (size_t)kChunk * (D + 1);
-    static constexpr size_t ph = (size_t)D * D;
+    static constexpr size_t ph = (size_t)D * (D + 1);   // phi^T, rows padded (no bank conflicts)
     static constexpr size_t region = (xs + ph) > ((size_t)kChunk * kChunk + (size_t)kChunk * 2 * D)
                                          ? (xs + ph)
                                          : ((size_t)kChunk * kChunk + (size_t)kChunk * 2 * D);
@@ -83,7 +83,7 @@ __device__ __forceinline__ void project(const TIO* __restrict__ x, const TIO* __
     const TIO* ph = phi + (size_t)h * D * D;
     for (int e = tid; e < D * D; e += kThreads) {
         const int o = e / D, i = e % D;
-        Ph[i * D + o] = to_f32(ph[e]);  // phi^T
+        Ph[i * (D + 1) + o] = to_f32(ph[e]);  // phi^T
     }
     __syncthreads();
     constexpr int CT = D / 16;           // columns per thread
@@ -98,7 +98,7 @@ __device__ __forceinline__ void project(const TIO* __restrict__ x, const TIO* __
 #pragma unroll
         for (int r = 0; r < 4; ++r) xr[r] = Xs[(tg * 4 + r) * (D + 1) + i];
 #pragma unroll
-        for (int c = 0; c < CT; ++c) pc[c] = Ph[i * D + og + 16 * c];
+        for (int c = 0; c < CT; ++c) pc[c] = Ph[i * (D + 1) + og + 16 * c];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -184,28 +184,53 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
     }
     __syncthreads();
     // L (strictly lower, decayed, beta-scaled k'.k') and the masked decayed q'.k':
-    // a warp per pair (t, s), its lanes over the feature index
-    for (int e = warp; e < kChunk * kChunk; e += kThreads / 32) {
-        const int t = e / kChunk, s = e % kChunk;
-        float l = 0.f, qk = 0.f;
-        if (s < t) {
-            float dk = 0.f, dq = 0.f;
+    // two 64 x 64 products over the features, from a transposed copy of K' (in
+    // the projections' staging space, free now)
+    {
+        float* KT = sm + P::xs;  // [D][C]
+        for (int e = tid; e < kChunk * D; e += kThreads) {
+            const int t = e / D, i = e % D;
+            KT[i * kChunk + t] = Kp[e];
+        }
+        __syncthreads();
+        const int tg = tid / 16, sg = tid % 16;  // rows 4 tg..+3, columns sg + 16 c
+        float dk[4][4], dq[4][4];
 #pragma unroll
-            for (int i = lane; i < D; i += 32) {
-                const float ks = Kp[s * D + i];
-                dk = fmaf(Kp[t * D + i], ks, dk);
-                dq = fmaf(Qp[t * D + i], ks, dq);
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dk[r][c] = dq[r][c] = 0.f;
+        for (int i = 0; i < D; ++i) {
+            float kr[4], qr[4], ks[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                kr[r] = Kp[(tg * 4 + r) * D + i];
+                qr[r] = Qp[(tg * 4 + r) * D + i];
             }
-            dk = warp_sum(dk);
-            dq = warp_sum(dq);
-            const float dd = expf(fminf(lam[t - 1] - lam[s], 0.f));
-            l = bet[t] * dd * dk;
-            qk = dd * dq;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ks[c] = KT[i * kChunk + sg + 16 * c];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    dk[r][c] = fmaf(kr[r], ks[c], dk[r][c]);
+                    dq[r][c] = fmaf(qr[r], ks[c], dq[r][c]);
+                }
         }
-        if (lane == 0) {
-            Ls[e] = l;
-            rec[R::QK + e] = qk;
-        }
+        __syncthreads();  // KT is overwritten by L below
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int t = tg * 4 + r, s2 = sg + 16 * c;
+                float l = 0.f, qk = 0.f;
+                if (s2 < t) {
+                    const float dd = expf(fminf(lam[t - 1] - lam[s2], 0.f));
+                    l = bet[t] * dd * dk[r][c];
+                    qk = dd * dq[r][c];
+                }
+                Ls[t * kChunk + s2] = l;
+                rec[R::QK + t * kChunk + s2] = qk;
+            }
     }
     // right-hand sides [beta V' | beta gprev K'] and the forward substitution,
     // one column per thread
@@ -270,7 +295,7 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
 #pragma unroll
             for (int q = 0; q < EI; ++q) {
                 const int i = ig + 16 * p, j = jg + 16 * q;
-                rec[R::M + (size_t)i * D + j] = (i == j ? gend : 0.f) - m[p][q];
+                rec[R::M + (size_t)j * D + i] = (i == j ? gend : 0.f) - m[p][q];  // stored transposed
                 rec[R::N + (size_t)i * D + j] = nn[p][q];
             }
     }
@@ -280,56 +305,74 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(LayerArgs a, float
 // every chunk's start state is saved for the reads, S_N goes to the state.
 template <int D>
 struct ChainSmem {
-    // M with rows padded to D + 1 floats (thread i reads row i: no bank conflicts)
-    static constexpr size_t bytes = sizeof(float) * ((size_t)D * (D + 1) + (size_t)D * kBand);
+    // two M^T buffers (bulk copies, double-buffered), the band of S, two mbarriers
+    static constexpr size_t bytes = sizeof(float) * (2 * (size_t)D * D + (size_t)D * kBand) + 64;
 };
 
+// S_{c+1} = M_c S_c + N_c over the chunks of one head, for kBand columns of S;
+// every chunk's start state is saved for the reads, S_N goes to the state.
+// M_{c+1}^T is copied into shared memory (one bulk copy) while step c runs.
 template <int D>
 __global__ void __launch_bounds__(D) chunk_chain_kernel(LayerArgs a, float* __restrict__ rec_base) {
     using R = Rec<D>;
-    extern __shared__ __align__(16) float csm[];
-    float* Ms = csm;                                   // [D][D + 1]
-    float (*Ss)[kBand] = reinterpret_cast<float (*)[kBand]>(csm + (size_t)D * (D + 1));
+    extern __shared__ __align__(128) float csm[];
+    float* MT = csm;                                                  // [2][D][D]
+    float (*Ss)[kBand] = reinterpret_cast<float (*)[kBand]>(csm + 2 * (size_t)D * D);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(csm + 2 * (size_t)D * D + (size_t)D * kBand);
+    volatile int* abort_word = reinterpret_cast<volatile int*>(bar + 2);
     const int band = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int j0 = band * kBand;
     const int i = threadIdx.x;  // row of S
     const size_t bh = (size_t)b * a.H + h;
     const int nch = (a.T + kChunk - 1) / kChunk;
     float* S = a.state + bh * D * D;
+    constexpr uint32_t kMBytes = (uint32_t)(D * D * sizeof(float));
+    if (i == 0) {
+        sm100::mbar_init(&bar[0], 1);
+        sm100::mbar_init(&bar[1], 1);
+        *abort_word = 0;
+        sm100::fence_mbar_init();
+        sm100::mbar_expect_tx(&bar[0], kMBytes);
+        sm100::bulk_load(sm100::smem_u32(MT), rec_base + (bh * nch) * R::floats + R::M, kMBytes, &bar[0]);
+    }
+    __syncthreads();
     float s[kBand];
 #pragma unroll
     for (int j = 0; j < kBand; ++j) s[j] = S[(size_t)i * D + j0 + j];
+    bool ok = true;
     for (int c = 0; c < nch; ++c) {
         float* rec = rec_base + (bh * nch + c) * R::floats;
+        const int buf = c & 1;
+        if (i == 0 && c + 1 < nch) {
+            // the other buffer was last read in step c - 1 (every thread passed the
+            // barrier at its end): M_{c+1}^T goes there
+            sm100::mbar_expect_tx(&bar[buf ^ 1], kMBytes);
+            sm100::bulk_load(sm100::smem_u32(MT + (size_t)(buf ^ 1) * D * D), rec + R::floats + R::M, kMBytes,
+                             &bar[buf ^ 1]);
+        }
 #pragma unroll
         for (int j = 0; j < kBand; ++j) {
             rec[R::S0 + (size_t)i * D + j0 + j] = s[j];
             Ss[i][j] = s[j];
         }
-        const float4* M4 = reinterpret_cast<const float4*>(rec + R::M);
-        for (int e = i; e < D * D / 4; e += D) {
-            const float4 v = M4[e];
-            const int r = (4 * e) / D, cc = (4 * e) % D;
-            float* dst = Ms + r * (D + 1) + cc;
-            dst[0] = v.x;
-            dst[1] = v.y;
-            dst[2] = v.z;
-            dst[3] = v.w;
-        }
-        __syncthreads();
         float acc[kBand];
 #pragma unroll
         for (int j = 0; j < kBand; ++j) acc[j] = rec[R::N + (size_t)i * D + j0 + j];
-        for (int k = 0; k < D; ++k) {
-            const float mik = Ms[i * (D + 1) + k];
+        ok = ok && sm100::mbar_wait(&bar[buf], (c >> 1) & 1, abort_word, a.flags, a.wait_ns);
+        __syncthreads();
+        if (ok) {
+            const float* Mb = MT + (size_t)buf * D * D;
+            for (int k = 0; k < D; ++k) {
+                const float mik = Mb[k * D + i];
 #pragma unroll
-            for (int j = 0; j < kBand; ++j) acc[j] = fmaf(mik, Ss[k][j], acc[j]);
+                for (int j = 0; j < kBand; ++j) acc[j] = fmaf(mik, Ss[k][j], acc[j]);
+            }
         }
 #pragma unroll
         for (int j = 0; j < kBand; ++j) s[j] = acc[j];
         __syncthreads();
     }
-    bool bad = false;
+    bool bad = !ok;
 #pragma unroll
     for (int j = 0; j < kBand; ++j) {
         S[(size_t)i * D + j0 + j] = s[j];
