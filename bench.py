@@ -54,9 +54,11 @@ def _args():
     p.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     p.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--layer", choices=["hybrid", "kvcache"], default="hybrid",
+    p.add_argument("--layer", choices=["hybrid", "kvcache", "token", "tra"], default="hybrid",
                    help="hybrid: the ARL2 layer (the reported benchmark); kvcache: the softmax "
-                        "baseline with a growing key/value cache on the same stream, for comparison")
+                        "baseline with a growing key/value cache on the same stream, for comparison; "
+                        "token: the token-level access variant; tra: Token Radius Attention on the "
+                        "intra-frame branch against the dense layer")
     p.add_argument("--workload", choices=["480p", "720p", "stream14b", "long"], default="480p",
                    help="480p: the reported benchmark (21 frames of 1560 tokens, H12); 720p: 21 frames "
                         "of 3600 tokens, H40; stream14b: one frame of the Wan-14B shape (H40) as 4 "
@@ -612,6 +614,135 @@ def run_kvcache(args):
     return 0
 
 
+def run_token(args):
+    """The token-level access variant on the 480p stream (21 frames, one clean pass
+    each, inputs resident), beside the frame-level layer: time per frame from CUDA
+    events around the whole stream, per-kernel times from the timing hook."""
+    import torch
+    import gated_delta_linear_b200 as G
+    import workloads as W
+
+    w = W.WORKLOADS[1]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    phi = W.feature_maps(w)
+    fr = [[t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)]
+          for x in (W.pass_inputs(w, n, 0) for n in range(w.frames))]
+    out = torch.empty_like(fr[0][0])
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, cls in (("token_level", G.TokenLevelAttention), ("frame_level", G.HybridAttention)):
+        L = cls(w.B, w.H, w.T, w.d, w.torch_dtype, *phi, device=dev)
+
+        def step():
+            L.state.zero_()
+            for f in fr:
+                L.forward(*f, 1, out=out)
+
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = max(2, args.steps // 50)
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        assert G.hyb_attn_timing_begin(w.frames * 8 + 8) == G.HYB_OK
+        step()
+        torch.cuda.synchronize(dev)
+        st, per, _ = G.hyb_attn_timing_end()
+        res[name] = {"us_per_frame": a.elapsed_time(b) / steps / w.frames * 1e3,
+                     "kernel_us_per_launch": {k: v[1] / v[0] * 1e3 for k, v in per.items() if v[0]},
+                     "device_status": G.hyb_attn_status_string(L.device_status())}
+    tok = res["token_level"]["us_per_frame"]
+    # the method's algorithmic work per token and head: 4 T d (intra) + 12 d^2
+    # (three 1x1 maps, the read q'S, and the token's update k'^T S and k (v - ...)^T)
+    flops = w.B * w.H * w.T * (4.0 * w.T * w.d + 12.0 * w.d * w.d)
+    line = {"layer": "token_level_access", "metric": "hybrid-attn layer tokens/s, token-level access "
+            "(21-frame 480p forward, 1 B200)", "unit": "tokens/s", "value": w.B * w.T / (tok / 1e6),
+            "us_per_frame": tok, "frame_level_us_per_frame": res["frame_level"]["us_per_frame"],
+            "achieved_tflops": flops / (tok / 1e6) / 1e12, "higher_is_better": True, "dtype": "bf16 I/O, fp32 chunked recurrence",
+            "data": "synthetic (seeded normals, video-DiT shapes)", **res}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tra(args):
+    """Token Radius Attention on the 480p shape (B1 H12, 30 x 52 patches in tiles of
+    8 x 16, tau 0.15, two votes), per frame as the page uses it across denoising
+    steps: one dense warm-up pass (query-only) that writes the entropies, then three
+    query-only and one clean pass that attend over the kept key blocks; timed
+    against the same five passes all dense.  Inputs resident; CUDA events."""
+    import torch
+    import gated_delta_linear_b200 as G
+    import workloads as W
+
+    w = W.WORKLOADS[1]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    frames = 6
+    desc = G.make_desc(w.B, w.H, w.T, w.d, G.HYB_BF16)
+    params = G.HybTraParams(30, 52, 8, 16, 0.15, 2)
+    phi = [p.to(dev) for p in W.feature_maps(w)]
+    ins = []
+    for n in range(frames):
+        per = []
+        for p in range(5):
+            x = W.pass_inputs(w, n, p)
+            per.append([t.to(dev) for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits)])
+        ins.append(per)
+    out = torch.empty_like(ins[0][0][0])
+    ent = torch.zeros(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+    ws = torch.zeros(G.hyb_tra_workspace_bytes(desc), dtype=torch.uint8, device=dev)
+    S = torch.zeros(w.B, w.H, w.d, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def tra_step():
+        S.zero_()
+        for per in ins:
+            assert G.hyb_tra_forward(desc, params, 1, *per[0][:3], *phi, *per[0][3:], S, 0, out, ent, ws) == 0
+            for p in range(1, 5):
+                assert G.hyb_tra_forward(desc, params, 0, *per[p][:3], *phi, *per[p][3:], S, int(p == 4), out, ent,
+                                         ws) == 0
+
+    def dense_step():
+        S.zero_()
+        for per in ins:
+            for p in range(5):
+                assert G.hyb_attn_forward(desc, *per[p][:3], *phi, *per[p][3:], S, int(p == 4), out, ws) == 0
+
+    res = {}
+    for name, fn in (("tra", tra_step), ("dense", dense_step)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = max(3, args.steps // 20)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = a.elapsed_time(b) / steps / frames * 1e3
+    # retained key blocks of the last sparse pass (the lists sit after the pass's workspace)
+    nkb = (w.T + 127) // 128
+    base = (G.hyb_attn_workspace_bytes(desc) + 255) // 256 * 256
+    lists = (w.B * w.H * nkb * nkb * 4 + 255) // 256 * 256
+    counts = ws[base + lists: base + lists + w.B * w.H * nkb * 4].view(torch.int32)
+    retained = float(counts.double().sum().item()) / (w.B * w.H * nkb * nkb)
+    line = {"layer": "token_radius_attention", "metric": "hybrid-attn layer us per frame, 5 passes per frame "
+            "(1 dense warm-up + 4 block-sparse), 480p shape, 1 B200", "unit": "us/frame", "value": res["tra"],
+            "dense_us_per_frame": res["dense"], "speedup_vs_dense": res["dense"] / res["tra"],
+            "retained_key_blocks": retained, "frames": frames, "higher_is_better": False, "dtype": "bf16",
+            "data": "synthetic (seeded normals, 480p shape, tile-major order by construction)",
+            "config": {"B": w.B, "H": w.H, "T": w.T, "grid": [30, 52], "tiles": [8, 16], "tau": 0.15,
+                       "votes_min": 2}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_long(args):
     """The long-stream workload (B=2, H=12, 240 frames of 1560 tokens, a pool of
     8 frames cycled), once with the state carried through the stream (the literal
@@ -699,6 +830,10 @@ def main():
         return run_reference(args)
     if args.layer == "kvcache":
         return run_kvcache(args)
+    if args.layer == "tra":
+        return run_tra(args)
+    if args.layer == "token":
+        return run_token(args)
     if args.workload == "long":
         return run_long(args)
     if args.workload != "480p" and args.gpus > 1:

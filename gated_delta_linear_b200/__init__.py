@@ -36,6 +36,9 @@ from ._binding import (  # noqa: F401
     TokenLevelAttention,
     hyb_attn_forward_token_level,
     hyb_attn_forward_frames,
+    HybTraParams,
+    hyb_tra_forward,
+    hyb_tra_workspace_bytes,
     hyb_attn_frames_workspace_bytes,
     hyb_attn_token_level_workspace_bytes,
     KVCacheAttention,

@@ -35,6 +35,11 @@ class HybAttnDesc(ctypes.Structure):
     ]
 
 
+class HybTraParams(ctypes.Structure):
+    _fields_ = [("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("tile_h", ctypes.c_int),
+                ("tile_w", ctypes.c_int), ("tau", ctypes.c_float), ("votes_min", ctypes.c_int)]
+
+
 HYB_NUM_KERNELS = 7
 
 
@@ -62,6 +67,11 @@ def _load():
     L.hyb_attn_forward_noalloc.restype = i
     L.hyb_attn_forward_mixed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.hyb_attn_forward_mixed.restype = i
+    L.hyb_tra_workspace_bytes.argtypes = [dp]
+    L.hyb_tra_workspace_bytes.restype = sz
+    L.hyb_tra_forward.argtypes = [dp, ctypes.POINTER(HybTraParams), i, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp,
+                                  vp, vp, sz, vp]
+    L.hyb_tra_forward.restype = i
     L.hyb_attn_frames_workspace_bytes.argtypes = [dp, i]
     L.hyb_attn_frames_workspace_bytes.restype = sz
     L.hyb_attn_forward_frames.argtypes = [dp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -148,6 +158,22 @@ def hyb_attn_forward_noalloc(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, be
                                         _ptr(phi_q), _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits),
                                         _ptr(beta_logits), _ptr(state), int(clean_pass), _ptr(out),
                                         _stream(stream))
+
+
+def hyb_tra_workspace_bytes(desc: HybAttnDesc) -> int:
+    return lib.hyb_tra_workspace_bytes(ctypes.byref(desc))
+
+
+def hyb_tra_forward(desc, params, warmup, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                    clean_pass, out, entropy, workspace, workspace_bytes=None, stream=None) -> int:
+    """Token Radius Attention pass: warmup=1 is the dense pass that also writes the
+    per-query entropies; warmup=0 attends over the key blocks those entropies keep."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_tra_forward(ctypes.byref(desc), ctypes.byref(params), int(warmup), _ptr(q), _ptr(k), _ptr(v),
+                               _ptr(phi_q), _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits), _ptr(beta_logits),
+                               _ptr(state), int(clean_pass), _ptr(out), _ptr(entropy), _ptr(workspace),
+                               workspace_bytes, _stream(stream))
 
 
 def hyb_attn_frames_workspace_bytes(desc: HybAttnDesc, n_frames: int) -> int:

@@ -48,6 +48,13 @@ struct LayerArgs {
     // token-level access: the inter-frame read computed by the token-level kernels,
     // fp32 [B][T][H][D]; the attention kernels add it instead of Q W (NULL: Q W)
     const float* oi_ext;
+    // Token Radius Attention: the warm-up pass writes each query's attention entropy
+    // (nats, [B][H][T]); a sparse pass walks, for query tile qt of (b, h), the
+    // kv_count[bh * n_qt + qt] key blocks listed at kv_list[(bh * n_qt + qt) * kv_stride]
+    float* ent_out;
+    const int* kv_list;
+    const int* kv_count;
+    int kv_stride;
     // bounded device waits give up after wait_ns (2 s unless a fault test shortens it)
     unsigned long long wait_ns;
     int dbg_skip_v;            // fault test only: the attention kernel's V producer issues nothing

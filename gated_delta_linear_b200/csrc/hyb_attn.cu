@@ -16,6 +16,7 @@
 #include "tc_kernels.cuh"
 #include "tc_attention.cuh"
 #include "token_level.cuh"
+#include "tra.cuh"
 
 namespace {
 
@@ -239,7 +240,9 @@ struct TcPass {
         a = args;
         cudaError_t e;
         if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
-        if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+        static unsigned char done_attn_ent[kMaxDevices];
+        if ((e = opt_in_smem(tc::attention_kernel<false>, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::attention_kernel<true>, tc::attn::SMEM, done_attn_ent)) != cudaSuccess) return e;
         if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
         const uint64_t row_bytes = (uint64_t)a.H * D * 2;
         const uint64_t bh = (uint64_t)a.B * a.H;
@@ -286,8 +289,10 @@ struct TcPass {
         cfg.attrs = at;
         cfg.numAttrs = pdl ? 1 : 0;
         cudaError_t le = cudaSuccess;
+        // the entropy-writing variant for the warm-up pass of Token Radius Attention
         cudaError_t e = timed(K_ATTN, st, [&] {
-            le = cudaLaunchKernelEx(&cfg, tc::attention_kernel, a, tq, tk, tv, tw, tout);
+            le = a.ent_out ? cudaLaunchKernelEx(&cfg, tc::attention_kernel<true>, a, tq, tk, tv, tw, tout)
+                           : cudaLaunchKernelEx(&cfg, tc::attention_kernel<false>, a, tq, tk, tv, tw, tout);
         });
         return e != cudaSuccess ? e : le;
     }
@@ -436,7 +441,7 @@ cudaError_t launch_token_level(LayerArgs a, const TokPlan& tp, char* ws, cudaStr
     a.oi_ext = oi;
     if constexpr (D == 128) {
         static unsigned char done_attn[kMaxDevices];
-        if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::attention_kernel<false>, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
         const uint64_t row_bytes = (uint64_t)a.H * D * 2;
         CUtensorMap tq, tk, tv, tout;
         if (!map3d(&tq, a.q, (uint64_t)a.H * D, a.T, a.B, row_bytes, row_bytes * a.T) ||
@@ -453,7 +458,7 @@ cudaError_t launch_token_level(LayerArgs a, const TokPlan& tp, char* ws, cudaStr
         cudaError_t le = cudaSuccess;
         // tq stands in for the unused W map
         e = timed(K_ATTN, st,
-                  [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
+                  [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel<false>, a, tq, tk, tv, tq, tout); });
         if (e != cudaSuccess) return e;
         if (le != cudaSuccess) return le;
     } else {
@@ -604,7 +609,7 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
 
     static unsigned char done_attn[kMaxDevices];
     cudaError_t e;
-    if ((e = opt_in_smem(tc::attention_kernel, tc::attn::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
+    if ((e = opt_in_smem(tc::attention_kernel<false>, tc::attn::SMEM, done_attn)) != cudaSuccess) return HYB_ERR_CUDA;
     const uint64_t row_bytes = (uint64_t)H * D * 2;
     CUtensorMap tq, tk, tv, tout;
     if (!map3d(&tq, q, (uint64_t)H * D, T, B, row_bytes, row_bytes * T) ||
@@ -619,7 +624,7 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     acfg.stream = st;
     cudaError_t le = cudaSuccess;
     // tq stands in for the unused W map
-    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel, a, tq, tk, tv, tq, tout); });
+    e = timed(K_ATTN, st, [&] { le = cudaLaunchKernelEx(&acfg, tc::attention_kernel<false>, a, tq, tk, tv, tq, tout); });
     if (e != cudaSuccess || le != cudaSuccess) return HYB_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
@@ -669,6 +674,63 @@ hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc, const void* q, cons
     if (!mix || !out) return HYB_ERR_INVALID;
     return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out,
                         nullptr, nullptr, workspace, workspace_bytes, stream, mix);
+}
+
+// ---- Token Radius Attention ------------------------------------------------------
+static bool tra_params_ok(const hyb_attn_desc* d, const hyb_tra_params* p) {
+    return p && p->grid_h > 0 && p->grid_w > 0 && p->grid_h < 32768 && p->grid_w < 32768 &&
+           (long long)p->grid_h * p->grid_w == d->T && p->tile_h > 0 && p->tile_w > 0 && p->votes_min >= 1 &&
+           p->tau > 0.f && isfinite(p->tau);
+}
+
+size_t hyb_tra_workspace_bytes(const hyb_attn_desc* desc) {
+    Plan p;
+    if (make_plan(desc, &p) != HYB_OK || !p.bf16) return 0;
+    const size_t nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
+    const size_t bh = (size_t)desc->B * desc->H;
+    return align_up(align_up(p.total, 256) + bh * nkb * nkb * sizeof(int), 256) + align_up(bh * nkb * sizeof(int), 256);
+}
+
+hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* params, int warmup, const void* q,
+                           const void* k, const void* v, const void* phi_q, const void* phi_k, const void* phi_v,
+                           const float* gate_logits, const float* beta_logits, float* state, int clean_pass,
+                           void* out, float* entropy, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!out || !entropy) return HYB_ERR_INVALID;
+    Plan p;
+    hyb_status s = make_plan(desc, &p);
+    if (s != HYB_OK) return s;
+    if (!p.bf16) return HYB_ERR_UNSUPPORTED;
+    if (!tra_params_ok(desc, params) || (warmup != 0 && warmup != 1)) return HYB_ERR_INVALID;
+    if (((uintptr_t)entropy & 15u) != 0) return HYB_ERR_ALIGN;
+    const size_t need = hyb_tra_workspace_bytes(desc);
+    if (!workspace || workspace_bytes < need) return HYB_ERR_WORKSPACE;
+    LayerArgs a;
+    s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out, nullptr,
+                  nullptr, workspace, workspace_bytes, nullptr, &a, &p);
+    if (s != HYB_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (warmup) {
+        // dense pass; the attention kernel also writes every query's entropy
+        a.ent_out = entropy;
+        return launch_tc(a, clean_pass, st) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+    }
+    const int nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
+    int* list = (int*)((char*)workspace + align_up(p.total, 256));
+    int* count = (int*)((char*)list + align_up((size_t)desc->B * desc->H * nkb * nkb * sizeof(int), 256));
+    static unsigned char done_mask[kMaxDevices];
+    const size_t msm = tra::mask_smem_bytes(nkb);
+    if (msm > 227u * 1024u) return HYB_ERR_UNSUPPORTED;
+    cudaError_t e = opt_in_smem(tra::mask_kernel, msm, done_mask);
+    if (e != cudaSuccess) return HYB_ERR_CUDA;
+    const tra::Params tp = {params->grid_h, params->grid_w, params->tile_h, params->tile_w, params->tau,
+                            params->votes_min};
+    tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kBlock, msm, st>>>(a, tp, entropy, list, count);
+    if ((e = cudaGetLastError()) != cudaSuccess) return HYB_ERR_CUDA;
+    // block-sparse pass: the attention kernel walks the kept key blocks
+    a.kv_list = list;
+    a.kv_count = count;
+    a.kv_stride = nkb;
+    return launch_tc(a, clean_pass, st) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
 size_t hyb_attn_frames_workspace_bytes(const hyb_attn_desc* desc, int n_frames) {

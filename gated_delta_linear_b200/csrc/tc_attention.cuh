@@ -83,6 +83,30 @@ __device__ __forceinline__ float exp_scores(const float* x, float scale, float n
     return (l4[0] + l4[1]) + (l4[2] + l4[3]);
 }
 
+// The same with the row's sum of p (y - m) in *A (y = x * scale), for the
+// attention entropy; masked scores (-inf) give p = 0 and add nothing.
+template <int N>
+__device__ __forceinline__ float exp_scores_ent(const float* x, float scale, float neg_m, uint32_t* pk, float* A) {
+    float l4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < N / 2; ++k) {
+        const float t0 = fmaxf(fmaf(x[2 * k], scale, neg_m), -1e30f);
+        const float t1 = fmaxf(fmaf(x[2 * k + 1], scale, neg_m), -1e30f);
+        const float e0 = ex2(t0), e1 = ex2(t1);
+        l4[(2 * k) & 3] += e0;
+        l4[(2 * k + 1) & 3] += e1;
+        a4[(2 * k) & 3] = fmaf(e0, t0, a4[(2 * k) & 3]);
+        a4[(2 * k + 1) & 3] = fmaf(e1, t1, a4[(2 * k + 1) & 3]);
+        pk[k] = pack_bf16(e0, e1);
+    }
+    *A = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    return (l4[0] + l4[1]) + (l4[2] + l4[3]);
+}
+
+// kEnt: the warm-up pass of Token Radius Attention, which also writes each
+// query's attention entropy (a.ent_out).  A key-block list (a.kv_list) makes
+// the key loop walk only the listed blocks (block-sparse intra-frame attention).
+template <bool kEnt>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     attention_kernel(const __grid_constant__ LayerArgs a, const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -108,9 +132,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T;
     const int q0 = qt_ * kTile;
-    const int n = (a.T_kv + kTile - 1) / kTile;  // key tiles
+    const int bh_ = b * a.H + h;
+    const size_t kvrow = ((size_t)bh_ * gridDim.x + qt_);
+    // key tiles: every tile of the frame, or the listed ones (block-sparse)
+    const int n = a.kv_count ? a.kv_count[kvrow] : (a.T_kv + kTile - 1) / kTile;
+    const int* kvl = a.kv_list ? a.kv_list + kvrow * a.kv_stride : nullptr;
+    auto ktile = [&](int j) { return kvl ? kvl[j] : j; };  // frame tile of the j-th key tile walked
     const bool inter = a.inter != 0;             // add O_inter = Q W (hybrid layer)
-    const int bh = b * a.H + h;
+    const int bh = bh_;
     // K stages that receive W_hi / W_lo at the end (free once the scores of key
     // tiles n-3 / n-2 are computed; stages no tile uses when n is small)
     const int wst_hi = n >= 3 ? (n - 3) % kKStages : 2;
@@ -134,8 +163,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0, b);
         for (int j = 0; j < kKStages && j < n; ++j) {
             mbar_expect_tx(&bars[B_KFULL + j], kTileBytes);
-            tma_load_3d(sb + K0 + j * kTileBytes, &tm_k, &bars[B_KFULL + j], xh, j * kTile, b);
-            tma_load_3d(sb + K0 + j * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + j], xh + 64, j * kTile, b);
+            tma_load_3d(sb + K0 + j * kTileBytes, &tm_k, &bars[B_KFULL + j], xh, ktile(j) * kTile, b);
+            tma_load_3d(sb + K0 + j * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + j], xh + 64, ktile(j) * kTile, b);
         }
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
@@ -161,8 +190,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     !mbar_wait(&bars[B_VEMPTY + vs], ((j / kVStages) + 1) & 1, abort_word, a.flags, a.wait_ns))
                     break;
                 mbar_expect_tx(&bars[B_VFULL + vs], kTileBytes);
-                tma_load_3d(sb + V0 + vs * kTileBytes, &tm_v, &bars[B_VFULL + vs], xh, j * kTile, b);
-                tma_load_3d(sb + V0 + vs * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + vs], xh + 64, j * kTile, b);
+                tma_load_3d(sb + V0 + vs * kTileBytes, &tm_v, &bars[B_VFULL + vs], xh, ktile(j) * kTile, b);
+                tma_load_3d(sb + V0 + vs * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + vs], xh + 64, ktile(j) * kTile,
+                            b);
             }
         }
         __syncwarp();
@@ -177,8 +207,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 const int ks = j % kKStages;
                 if (!(ok = mbar_wait(&bars[B_KEMPTY + ks], ((j / kKStages) + 1) & 1, abort_word, a.flags, a.wait_ns))) break;
                 mbar_expect_tx(&bars[B_KFULL + ks], kTileBytes);
-                tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, j * kTile, b);
-                tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64, j * kTile, b);
+                tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, ktile(j) * kTile, b);
+                tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64, ktile(j) * kTile,
+                            b);
             }
             // W_hi / W_lo (row-major, MN-major operands) into K stages freed by S_{n-3} / S_{n-2}
             const int nbh = a.B * a.H;
@@ -300,6 +331,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const int mine = hf * 128 + r, theirs = (hf ^ 1) * 128 + r;  // + parity * 256
         const float scale = a.sm_scale_log2;
         float m = 0.f, l = 0.f;
+        float A = 0.f;  // kEnt: sum of p (y - m) over this half of the row
         float x[64];
         // this half of Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns));
@@ -333,7 +365,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&bars[B_SREAD + s]);  // S_j is in registers: S_{j+2} may overwrite it
-                const int valid = a.T_kv - j * kTile - (int)cs;
+                const int valid = a.T_kv - ktile(j) * kTile - (int)cs;
                 if (valid < 64) {
 #pragma unroll
                     for (int c = 0; c < 64; ++c)
@@ -348,8 +380,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 m = fmaxf(hm, xch[theirs]) * scale;
             }
             bool redo_h = false;
+            float At = 0.f;
             if (w_ok) {
-                lt = exp_scores<64>(x, scale, -m, pk);
+                lt = kEnt ? exp_scores_ent<64>(x, scale, -m, pk, &At) : exp_scores<64>(x, scale, -m, pk);
                 redo_h = !(lt < 9.2233720e18f);  // >= 2^63, inf or NaN
             }
             xfl[s * 256 + mine] = w_ok ? (redo_h ? 2 : 1) : 0;
@@ -358,7 +391,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             ok = __all_sync(0xffffffffu, w_ok && pc != 0);  // the same in both warps of the pair
             const bool redo = ok && (redo_h || pc == 2);
             const bool any_redo = __any_sync(0xffffffffu, redo);
-            float f = 1.0f;
+            float f = 1.0f, dm = 0.f;
             if (any_redo) {
                 // the offset is too low for this tile (or a score is not finite):
                 // move it to the row's max and redo P_j; O is rescaled below
@@ -368,11 +401,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 if (redo) {
                     const float mn = fmaxf(m, fmaxf(hm, xch[s * 256 + theirs]));
                     f = ex2(m - mn);
+                    dm = mn - m;
                     m = mn;
                 }
-                lt = exp_scores<64>(x, scale, -m, pk);
+                lt = kEnt ? exp_scores_ent<64>(x, scale, -m, pk, &At) : exp_scores<64>(x, scale, -m, pk);
             }
             if (!ok) continue;  // keep arriving at the pair barriers until the loop ends
+            // sum p (y - m) against the moved offset: f (A - dm l) (p scales by f)
+            if (kEnt) A = fmaf(f, A - dm * l, At);
             l = fmaf(l, f, lt);
             // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
             if (j > 0) {
@@ -415,11 +451,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // the pair barrier of tile n-1)
         xch[(n & 1) * 256 + mine] = l;
         xfl[(n & 1) * 256 + mine] = e_ok ? 1 : 0;
+        // kEnt: the halves' sums of p (y - m) through the K stage of tile n-1 (no
+        // product reads it any more; W lives in the stages of tiles n-3 and n-2)
+        float* xa = reinterpret_cast<float*>(smem + K0 + ((n - 1) % kKStages) * kTileBytes);
+        if (kEnt) xa[mine] = A;
         named_bar_sync(pair_bar, 64);
         const bool both = __all_sync(0xffffffffu, e_ok && xfl[(n & 1) * 256 + theirs] != 0);
         if (both) {
             tc_fence_after();
-            const float inv_l = 1.0f / (l + xch[(n & 1) * 256 + theirs]);  // commutative: the same in both halves
+            const float lrow_sum = l + xch[(n & 1) * 256 + theirs];
+            const float inv_l = 1.0f / lrow_sum;  // commutative: the same in both halves
+            if (kEnt && hf == 0 && q0 + r < T) {
+                // entropy (nats) of the row's softmax: ln l - ln 2 * sum p (y - m) / l
+                const float at = A + xa[theirs];
+                a.ent_out[(size_t)bh * T + q0 + r] = logf(lrow_sum) - 0.69314718f * at * inv_l;
+            }
             // out = a O_intra + O_inter (the inter gain c is folded into W); a = 1 without a mix
             const float inv_out = a.mix ? inv_l * a.mix[bh * 2] : inv_l;
             const int t = q0 + r;

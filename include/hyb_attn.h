@@ -217,6 +217,44 @@ hyb_status hyb_attn_forward_token_level(const hyb_attn_desc* desc,
                                         float* state, int clean_pass, void* out,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* hyb_tra_forward -- the hybrid layer with Token Radius Attention on its
+ * intra-frame branch ("Technical summary: Token Radius Attention",
+ * gist.science/ar/paper/2608.02504, §2): each query attends only to the key
+ * blocks near it on the frame's patch grid, with a radius set by its attention
+ * entropy.  warmup = 1: the dense pass of hyb_attn_forward (same outputs, same
+ * state update) that also writes every query's attention entropy
+ * H = -sum_j p_j ln p_j (nats) to `entropy` ([B][H][T] fp32, 16-byte aligned).
+ * warmup = 0: the entropies in `entropy` (from an earlier warm-up pass; the page
+ * reuses them across denoising steps) give each query a budget
+ * k = clamp(tau exp(H), 1, T) keys and a disk radius r = sqrt(k / pi) patches
+ * (the page's temporal decay exp(-gamma delta) is 1 on the current frame, the
+ * only one this branch attends to); a query votes for a key block when some key
+ * of it lies within r (Euclidean distance on patch coordinates); a key block is
+ * kept for a query block with at least votes_min votes, and always for itself;
+ * the intra-frame attention of each query then runs over the kept blocks of its
+ * query block (the block-sparse result).  The inter-frame read and the state
+ * update are those of hyb_attn_forward.  Blocks are runs of 128 tokens of the
+ * frame, which must be in tile-major order: tiles of tile_h x tile_w patches
+ * taken row-major over the grid_h x grid_w grid (grid_h * grid_w == T), patches
+ * row-major inside a tile, edge tiles cut by the grid; the caller orders q, k, v
+ * (and reads out) that way.  bf16 with d = 128 only (HYB_ERR_UNSUPPORTED
+ * otherwise).  workspace: hyb_tra_workspace_bytes(desc), zero-filled once.
+ * HYB_ERR_INVALID for bad params (grid sides >= 32768, tau <= 0 or not finite,
+ * votes_min < 1) or warmup outside {0, 1}; otherwise hyb_attn_forward's errors. */
+typedef struct {
+    int grid_h, grid_w;   /* the frame's patch grid (grid_h * grid_w == T) */
+    int tile_h, tile_w;   /* tile-major order */
+    float tau;            /* budget scale: k = tau exp(H) keys */
+    int votes_min;        /* votes that keep a key block (>= 1) */
+} hyb_tra_params;
+size_t hyb_tra_workspace_bytes(const hyb_attn_desc* desc);
+hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* params, int warmup,
+                           const void* q, const void* k, const void* v,
+                           const void* phi_q, const void* phi_k, const void* phi_v,
+                           const float* gate_logits, const float* beta_logits,
+                           float* state, int clean_pass, void* out, float* entropy,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* hyb_kvcache_attn_forward -- the softmax baseline the hybrid layer replaces
  * (ARL2 summary §1, problem statement: softmax self-attention whose key/value
  * cache grows with every generated chunk; §4, the memory and wall-clock

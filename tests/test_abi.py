@@ -134,3 +134,24 @@ def test_mixed_entry_requires_weights():
         == G.HYB_ERR_INVALID
     assert G.lib.hyb_attn_forward_mixed(ctypes.byref(d), *args, 1, FAKE + 8, FAKE, FAKE, 1 << 40, None) \
         == G.HYB_ERR_ALIGN
+
+
+def test_tra_host_validation_rejects_before_launch():
+    d = G.make_desc(1, 12, 1560, 128)
+    ok = G.HybTraParams(30, 52, 8, 16, 0.15, 2)
+    need = G.hyb_tra_workspace_bytes(d)
+    assert need > G.hyb_attn_workspace_bytes(d)
+    assert G.hyb_tra_workspace_bytes(G.make_desc(1, 2, 64, 32, G.HYB_FP32)) == 0
+
+    def call(params=ok, warmup=0, ent=FAKE, nbytes=need, desc=d):
+        return G.hyb_tra_forward(desc, params, warmup, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1,
+                                 FAKE, ent, FAKE, nbytes, 0)
+
+    assert call(params=G.HybTraParams(30, 51, 8, 16, 0.15, 2)) == G.HYB_ERR_INVALID   # grid != T
+    assert call(params=G.HybTraParams(30, 52, 8, 16, 0.0, 2)) == G.HYB_ERR_INVALID
+    assert call(params=G.HybTraParams(30, 52, 8, 16, 0.15, 0)) == G.HYB_ERR_INVALID
+    assert call(warmup=2) == G.HYB_ERR_INVALID
+    assert call(ent=None) == G.HYB_ERR_INVALID
+    assert call(ent=FAKE + 4) == G.HYB_ERR_ALIGN
+    assert call(nbytes=need - 1) == G.HYB_ERR_WORKSPACE
+    assert call(desc=G.make_desc(1, 2, 64, 32, G.HYB_FP32)) == G.HYB_ERR_UNSUPPORTED
