@@ -726,7 +726,8 @@ def run_tra(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         res[name] = a.elapsed_time(b) / steps / frames * 1e3
-    # retained key blocks of the last sparse pass (the lists sit after the pass's workspace)
+    # retained key blocks of the mask the last warm-up pass built (the lists sit after
+    # the pass's workspace)
     nkb = (w.T + 127) // 128
     base = (G.hyb_attn_workspace_bytes(desc) + 255) // 256 * 256
     lists = (w.B * w.H * nkb * nkb * 4 + 255) // 256 * 256

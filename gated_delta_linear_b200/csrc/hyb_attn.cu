@@ -709,24 +709,26 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
                   nullptr, workspace, workspace_bytes, nullptr, &a, &p);
     if (s != HYB_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (warmup) {
-        // dense pass; the attention kernel also writes every query's entropy
-        a.ent_out = entropy;
-        return launch_tc(a, clean_pass, st) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
-    }
     const int nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
     int* list = (int*)((char*)workspace + align_up(p.total, 256));
     int* count = (int*)((char*)list + align_up((size_t)desc->B * desc->H * nkb * nkb * sizeof(int), 256));
-    static unsigned char done_mask[kMaxDevices];
     const size_t msm = tra::mask_smem_bytes(nkb);
     if (msm > 227u * 1024u) return HYB_ERR_UNSUPPORTED;
-    cudaError_t e = opt_in_smem(tra::mask_kernel, msm, done_mask);
-    if (e != cudaSuccess) return HYB_ERR_CUDA;
-    const tra::Params tp = {params->grid_h, params->grid_w, params->tile_h, params->tile_w, params->tau,
-                            params->votes_min};
-    tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kBlock, msm, st>>>(a, tp, entropy, list, count);
-    if ((e = cudaGetLastError()) != cudaSuccess) return HYB_ERR_CUDA;
-    // block-sparse pass: the attention kernel walks the kept key blocks
+    if (warmup) {
+        // dense pass; the attention kernel also writes every query's entropy, then
+        // the block mask is built once from them (the later passes reuse it)
+        static unsigned char done_mask[kMaxDevices];
+        cudaError_t e = opt_in_smem(tra::mask_kernel, msm, done_mask);
+        if (e != cudaSuccess) return HYB_ERR_CUDA;
+        a.ent_out = entropy;
+        if (launch_tc(a, clean_pass, st) != cudaSuccess) return HYB_ERR_CUDA;
+        const tra::Params tp = {params->grid_h, params->grid_w, params->tile_h, params->tile_w, params->tau,
+                                params->votes_min};
+        tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kBlock, msm, st>>>(a, tp, entropy, list, count);
+        return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+    }
+    // block-sparse pass: the attention kernel walks the kept key blocks of the
+    // mask the last warm-up pass on this workspace built
     a.kv_list = list;
     a.kv_count = count;
     a.kv_stride = nkb;

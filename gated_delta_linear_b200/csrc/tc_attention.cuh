@@ -135,8 +135,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const int bh_ = b * a.H + h;
     const size_t kvrow = ((size_t)bh_ * gridDim.x + qt_);
     // key tiles: every tile of the frame, or the listed ones (block-sparse)
-    const int n = a.kv_count ? a.kv_count[kvrow] : (a.T_kv + kTile - 1) / kTile;
-    const int* kvl = a.kv_list ? a.kv_list + kvrow * a.kv_stride : nullptr;
+    // (a listed count of 0 means no mask has been built: every tile)
+    const int kvc = a.kv_count ? a.kv_count[kvrow] : 0;
+    const int n = kvc > 0 ? kvc : (a.T_kv + kTile - 1) / kTile;
+    const int* kvl = kvc > 0 ? a.kv_list + kvrow * a.kv_stride : nullptr;
     auto ktile = [&](int j) { return kvl ? kvl[j] : j; };  // frame tile of the j-th key tile walked
     const bool inter = a.inter != 0;             // add O_inter = Q W (hybrid layer)
     const int bh = bh_;

@@ -223,9 +223,12 @@ hyb_status hyb_attn_forward_token_level(const hyb_attn_desc* desc,
  * blocks near it on the frame's patch grid, with a radius set by its attention
  * entropy.  warmup = 1: the dense pass of hyb_attn_forward (same outputs, same
  * state update) that also writes every query's attention entropy
- * H = -sum_j p_j ln p_j (nats) to `entropy` ([B][H][T] fp32, 16-byte aligned).
- * warmup = 0: the entropies in `entropy` (from an earlier warm-up pass; the page
- * reuses them across denoising steps) give each query a budget
+ * H = -sum_j p_j ln p_j (nats) to `entropy` ([B][H][T] fp32, 16-byte aligned)
+ * and then builds the block mask from them in the workspace.  warmup = 0: the
+ * intra-frame attention runs block-sparse with the mask the last warm-up pass on
+ * this workspace built (the page computes the entropies once and reuses them
+ * across the later denoising steps; with no mask built yet the pass is dense;
+ * `entropy` is not read).  The mask: the entropies give each query a budget
  * k = clamp(tau exp(H), 1, T) keys and a disk radius r = sqrt(k / pi) patches
  * (the page's temporal decay exp(-gamma delta) is 1 on the current frame, the
  * only one this branch attends to); a query votes for a key block when some key
