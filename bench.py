@@ -733,10 +733,34 @@ def run_tra(args):
     lists = (w.B * w.H * nkb * nkb * 4 + 255) // 256 * 256
     counts = ws[base + lists: base + lists + w.B * w.H * nkb * 4].view(torch.int32)
     retained = float(counts.double().sum().item()) / (w.B * w.H * nkb * nkb)
+    max_kept = float(counts.max().item()) / nkb
+    # per-call times of each kind of pass (query-only, inputs of frame 0, the mask
+    # of the last warm-up kept for the sparse calls)
+    per0 = ins[0]
+    kinds = {
+        "warmup_with_mask": lambda: G.hyb_tra_forward(desc, params, 1, *per0[0][:3], *phi, *per0[0][3:], S, 0, out,
+                                                      ent, ws),
+        "sparse": lambda: G.hyb_tra_forward(desc, params, 0, *per0[1][:3], *phi, *per0[1][3:], S, 0, out, ent, ws),
+        "dense": lambda: G.hyb_attn_forward(desc, *per0[1][:3], *phi, *per0[1][3:], S, 0, out, ws),
+    }
+    per_call = {}
+    for name in ("warmup_with_mask", "dense", "sparse"):
+        fn = kinds[name]
+        for _ in range(3):
+            assert fn() == 0
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(50):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        per_call[name] = a.elapsed_time(b) / 50 * 1e3
     line = {"layer": "token_radius_attention", "metric": "hybrid-attn layer us per frame, 5 passes per frame "
             "(1 dense warm-up + 4 block-sparse), 480p shape, 1 B200", "unit": "us/frame", "value": res["tra"],
             "dense_us_per_frame": res["dense"], "speedup_vs_dense": res["dense"] / res["tra"],
-            "retained_key_blocks": retained, "frames": frames, "higher_is_better": False, "dtype": "bf16",
+            "retained_key_blocks": retained, "max_retained_per_query_block": max_kept,
+            "us_per_query_only_call": per_call, "frames": frames, "higher_is_better": False, "dtype": "bf16",
             "data": "synthetic (seeded normals, 480p shape, tile-major order by construction)",
             "config": {"B": w.B, "H": w.H, "T": w.T, "grid": [30, 52], "tiles": [8, 16], "tau": 0.15,
                        "votes_min": 2}}

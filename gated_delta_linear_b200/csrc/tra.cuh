@@ -48,43 +48,63 @@ __device__ __forceinline__ float radius2(float H, float tau, int T) {
     return fminf(fmaxf(tau * expf(H), 1.0f), (float)T) * 0.31830988618379067f;
 }
 
-// Shared memory: votes [nkb] ints, key-block boxes [nkb] int4, key positions [nkb * kBlock] ints.
+// Shared memory: key-block boxes [nkb] int4, run counts [nkb] ints, votes [nkb]
+// ints, runs [nkb * kBlock] int2.
 __host__ __device__ inline size_t mask_smem_bytes(int nkb) {
-    return (size_t)nkb * (sizeof(int) + sizeof(int4) + kBlock * sizeof(int));
+    return (size_t)nkb * (sizeof(int4) + 2 * sizeof(int) + kBlock * sizeof(int2));
 }
 
 // One CTA per (query block, head, batch), a thread per query of the block.
 // Writes the ascending list of kept key blocks of the query block at
 // list[(bh * nkb + qb) * nkb] and its length at count[bh * nkb + qb].
+//
+// A key block is described by its bounding box and by its runs: maximal
+// stretches of consecutive tokens on one patch row with consecutive columns
+// (a tile's row, or the part of it inside the block).  The distance from a
+// query to a run is exact (row offset and the column gap to the run's span),
+// so a query's vote needs one test per run instead of one per key; when the
+// block fills its box (a whole tile, or rows of one), the box test alone is
+// exact.  Decisions are those of the per-key test: the same integer squared
+// distances against the same fp32 squared radius.
 __global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, const float* __restrict__ ent,
                                                       int* __restrict__ list, int* __restrict__ count) {
     extern __shared__ __align__(16) unsigned char msm[];
     const int T = a.T;
     const int nkb = (T + kBlock - 1) / kBlock;
     int4* box = reinterpret_cast<int4*>(msm);                                 // (r0, r1, c0, c1)
-    int* kpos = reinterpret_cast<int*>(msm + (size_t)nkb * sizeof(int4));     // (r << 16) | c
-    int* votes = kpos + (size_t)nkb * kBlock;
+    int2* run = reinterpret_cast<int2*>(msm + (size_t)nkb * sizeof(int4));    // ((r << 16) | c0, c1)
+    int* nrun = reinterpret_cast<int*>(run + (size_t)nkb * kBlock);           // runs; -runs if the box is full
+    int* votes = nrun + nkb;
     const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
-    for (int j = tid; j < nkb * kBlock; j += kBlock) {
-        int r = 0, c = 0;
-        if (j < T) tile_major_pos(j, p, &r, &c);
-        kpos[j] = (r << 16) | c;
-    }
     for (int kb = tid; kb < nkb; kb += kBlock) votes[kb] = 0;
-    __syncthreads();
-    // bounding box of each key block's patches (a warp per block)
+    // runs and bounding box of each key block (a warp per block)
     for (int kb = warp; kb < nkb; kb += kBlock / 32) {
+        const int ntok = min(kBlock, T - kb * kBlock);
         int r0 = 1 << 30, r1 = -1, c0 = 1 << 30, c1 = -1;
-        for (int jj = lane; jj < kBlock; jj += 32) {
-            const int j = kb * kBlock + jj;
-            if (j >= T) break;
-            const int r = kpos[j] >> 16, c = kpos[j] & 0xffff;
-            r0 = min(r0, r);
-            r1 = max(r1, r);
-            c0 = min(c0, c);
-            c1 = max(c1, c);
+        int nstart = 0, nend = 0;
+        for (int base = 0; base < ntok; base += 32) {
+            const int i = base + lane, j = kb * kBlock + i;
+            const bool valid = i < ntok;
+            int r = 0, c = 0, rp = -1, cp = -2, rn = -1, cn = -2;
+            if (valid) {
+                tile_major_pos(j, p, &r, &c);
+                if (i > 0) tile_major_pos(j - 1, p, &rp, &cp);
+                if (i + 1 < ntok) tile_major_pos(j + 1, p, &rn, &cn);
+                r0 = min(r0, r);
+                r1 = max(r1, r);
+                c0 = min(c0, c);
+                c1 = max(c1, c);
+            }
+            const bool start = valid && !(rp == r && cp + 1 == c);
+            const bool end = valid && !(rn == r && cn == c + 1);
+            const unsigned ms = __ballot_sync(0xffffffffu, start), me = __ballot_sync(0xffffffffu, end);
+            const unsigned below = (1u << lane) - 1u;
+            if (start) run[kb * kBlock + nstart + __popc(ms & below)].x = (r << 16) | c;
+            if (end) run[kb * kBlock + nend + __popc(me & below)].y = c;
+            nstart += __popc(ms);
+            nend += __popc(me);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -93,25 +113,35 @@ __global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, con
             c0 = min(c0, __shfl_xor_sync(0xffffffffu, c0, o));
             c1 = max(c1, __shfl_xor_sync(0xffffffffu, c1, o));
         }
-        if (lane == 0) box[kb] = make_int4(r0, r1, c0, c1);
+        if (lane == 0) {
+            box[kb] = make_int4(r0, r1, c0, c1);
+            const bool full = (r1 - r0 + 1) * (c1 - c0 + 1) == ntok;
+            nrun[kb] = full ? -nstart : nstart;
+        }
     }
     __syncthreads();
     const int t = qb * kBlock + tid;
     const bool valid = t < T;
     const float r2 = valid ? radius2(ent[bh * T + t], p.tau, T) : -1.0f;
-    const int rq = valid ? kpos[t] >> 16 : 0, cq = valid ? kpos[t] & 0xffff : 0;
+    int rq = 0, cq = 0;
+    if (valid) tile_major_pos(t, p, &rq, &cq);
     for (int kb = 0; kb < nkb; ++kb) {
         const int4 bb = box[kb];
         const int dy = max(0, max(bb.x - rq, rq - bb.y)), dx = max(0, max(bb.z - cq, cq - bb.w));
         bool hit = false;
         if (valid && (float)(dy * dy + dx * dx) <= r2) {
-            for (int jj = 0; jj < kBlock; ++jj) {
-                const int j = kb * kBlock + jj;
-                if (j >= T) break;
-                const int ry = (kpos[j] >> 16) - rq, rx = (kpos[j] & 0xffff) - cq;
-                if ((float)(ry * ry + rx * rx) <= r2) {
-                    hit = true;
-                    break;
+            const int nr = nrun[kb];
+            if (nr < 0) {
+                hit = true;  // the block fills its box: the nearest point of the box is a key
+            } else {
+                for (int u = 0; u < nr; ++u) {
+                    const int2 ru = run[kb * kBlock + u];
+                    const int ry = (ru.x >> 16) - rq;
+                    const int rx = max(0, max((ru.x & 0xffff) - cq, cq - ru.y));
+                    if ((float)(ry * ry + rx * rx) <= r2) {
+                        hit = true;
+                        break;
+                    }
                 }
             }
         }

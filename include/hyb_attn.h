@@ -241,7 +241,9 @@ hyb_status hyb_attn_forward_token_level(const hyb_attn_desc* desc,
  * taken row-major over the grid_h x grid_w grid (grid_h * grid_w == T), patches
  * row-major inside a tile, edge tiles cut by the grid; the caller orders q, k, v
  * (and reads out) that way.  bf16 with d = 128 only (HYB_ERR_UNSUPPORTED
- * otherwise).  workspace: hyb_tra_workspace_bytes(desc), zero-filled once.
+ * otherwise) and T <= 28288 (221 key blocks: the mask kernel keeps every key
+ * block's bounding box and row runs in shared memory; HYB_ERR_UNSUPPORTED
+ * beyond).  workspace: hyb_tra_workspace_bytes(desc), zero-filled once.
  * HYB_ERR_INVALID for bad params (grid sides >= 32768, tau <= 0 or not finite,
  * votes_min < 1) or warmup outside {0, 1}; otherwise hyb_attn_forward's errors. */
 typedef struct {

@@ -155,3 +155,7 @@ def test_tra_host_validation_rejects_before_launch():
     assert call(ent=FAKE + 4) == G.HYB_ERR_ALIGN
     assert call(nbytes=need - 1) == G.HYB_ERR_WORKSPACE
     assert call(desc=G.make_desc(1, 2, 64, 32, G.HYB_FP32)) == G.HYB_ERR_UNSUPPORTED
+    # the mask kernel's shared memory holds at most 221 key blocks (T <= 28288)
+    big = G.make_desc(1, 1, 28289, 128)
+    assert call(desc=big, params=G.HybTraParams(1, 28289, 1, 16, 0.15, 2), nbytes=1 << 40) == \
+        G.HYB_ERR_UNSUPPORTED
