@@ -526,8 +526,8 @@ def run_cuda(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "api": ("hyb_attn_forward_frames (one call per 21-frame forward; bit-identical to one "
-                "hyb_attn_forward call per frame)") if frames_api else "hyb_attn_forward (one call per pass)",
+        "api": ("hyb_attn_forward_frames (one call per 21-frame forward: the kernels of one "
+                "hyb_attn_forward call per frame, scheduled over three streams)") if frames_api else "hyb_attn_forward (one call per pass)",
         "per_frame_calls": {"value": job_throughput(tokens_per_step, args.steps, world, ms_loop), "unit": UNIT,
                             "us_per_frame": 1e3 * ms_loop / args.steps / w.frames,
                             "api": "hyb_attn_forward, one call per pass (the autoregressive pattern)"},

@@ -55,6 +55,9 @@ struct LayerArgs {
     const int* kv_list;
     const int* kv_count;
     int kv_stride;
+    // optional: CTA i of the grid takes query tile row kv_order[i] (bh * n_qt + qt),
+    // so the longest lists go first
+    const int* kv_order;
     // bounded device waits give up after wait_ns (2 s unless a fault test shortens it)
     unsigned long long wait_ns;
     int dbg_skip_v;            // fault test only: the attention kernel's V producer issues nothing

@@ -34,6 +34,18 @@ struct Plan {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Token splits of the state update: about `want` splits of whole 128-token
+// tiles (at most one cluster's worth on the tensor path).
+void update_split(int T, int want, bool bf16, int* nsplit, int* split_tokens) {
+    const int ntiles = (T + kUpdateTile - 1) / kUpdateTile;
+    if (bf16 && want > tc::kMaxClusterRanks) want = tc::kMaxClusterRanks;
+    if (want > ntiles) want = ntiles;
+    if (want < 1) want = 1;
+    const int tiles_per_split = (ntiles + want - 1) / want;
+    *split_tokens = tiles_per_split * kUpdateTile;
+    *nsplit = (ntiles + tiles_per_split - 1) / tiles_per_split;
+}
+
 hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     if (!d) return HYB_ERR_INVALID;
     if (d->B <= 0 || d->H <= 0 || d->T <= 0 || d->d_k <= 0 || d->d_v <= 0) return HYB_ERR_INVALID;
@@ -53,15 +65,7 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     // distributed shared memory (no partials in the workspace).  fp32 path:
     // enough (b, h, split) blocks to cover the SMs, partials in the workspace.
     const int BH = d->B * d->H;
-    const int ntiles = (d->T + kUpdateTile - 1) / kUpdateTile;
-    int want = bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH;
-
-    if (bf16 && want > tc::kMaxClusterRanks) want = tc::kMaxClusterRanks;
-    if (want > ntiles) want = ntiles;
-    if (want < 1) want = 1;
-    const int tiles_per_split = (ntiles + want - 1) / want;
-    p->split_tokens = tiles_per_split * kUpdateTile;
-    p->nsplit = (ntiles + tiles_per_split - 1) / tiles_per_split;
+    update_split(d->T, bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
     const size_t hh = (size_t)BH * D * D;
     p->off_W = kStatusBytes;
     p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
@@ -486,10 +490,11 @@ hyb_status launch_pass(const LayerArgs& a, const Plan& p, int clean_pass, void* 
 // Per device: a high-priority stream for the state chain (prep, update of each
 // frame), a stream for the attention kernels, and events; created on the first
 // call on the device and kept.  The calls are not thread-safe.
+constexpr int kAttStreams = 2;  // attention kernels of consecutive frames alternate between them
 struct FrameRes {
     bool ready = false;
-    cudaStream_t chain = nullptr, att = nullptr;
-    cudaEvent_t fork = nullptr, join_chain = nullptr, join_att = nullptr;
+    cudaStream_t chain = nullptr, att[kAttStreams] = {};
+    cudaEvent_t fork = nullptr, join_chain = nullptr, join_att[kAttStreams] = {};
     cudaEvent_t* w = nullptr;
     int nw = 0;
 };
@@ -506,10 +511,12 @@ cudaError_t frame_resources(int n, FrameRes** out) {
         int least = 0, greatest = 0;
         if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
         if ((e = cudaStreamCreateWithPriority(&r.chain, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
-        if ((e = cudaStreamCreateWithPriority(&r.att, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+        for (int i = 0; i < kAttStreams; ++i) {
+            if ((e = cudaStreamCreateWithPriority(&r.att[i], cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+            if ((e = cudaEventCreateWithFlags(&r.join_att[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+        }
         if ((e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
         if ((e = cudaEventCreateWithFlags(&r.join_chain, cudaEventDisableTiming)) != cudaSuccess) return e;
-        if ((e = cudaEventCreateWithFlags(&r.join_att, cudaEventDisableTiming)) != cudaSuccess) return e;
         r.ready = true;
     }
     if (r.nw < n) {
@@ -688,7 +695,9 @@ size_t hyb_tra_workspace_bytes(const hyb_attn_desc* desc) {
     if (make_plan(desc, &p) != HYB_OK || !p.bf16) return 0;
     const size_t nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
     const size_t bh = (size_t)desc->B * desc->H;
-    return align_up(align_up(p.total, 256) + bh * nkb * nkb * sizeof(int), 256) + align_up(bh * nkb * sizeof(int), 256);
+    // block lists, their lengths, the schedule of the block-sparse grid
+    return align_up(align_up(p.total, 256) + bh * nkb * nkb * sizeof(int), 256) +
+           2 * align_up(bh * nkb * sizeof(int), 256);
 }
 
 hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* params, int warmup, const void* q,
@@ -712,6 +721,7 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
     const int nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
     int* list = (int*)((char*)workspace + align_up(p.total, 256));
     int* count = (int*)((char*)list + align_up((size_t)desc->B * desc->H * nkb * nkb * sizeof(int), 256));
+    int* order = (int*)((char*)count + align_up((size_t)desc->B * desc->H * nkb * sizeof(int), 256));
     const size_t msm = tra::mask_smem_bytes(nkb);
     if (msm > 227u * 1024u) return HYB_ERR_UNSUPPORTED;
     if (warmup) {
@@ -724,7 +734,9 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
         if (launch_tc(a, clean_pass, st) != cudaSuccess) return HYB_ERR_CUDA;
         const tra::Params tp = {params->grid_h, params->grid_w, params->tile_h, params->tile_w, params->tau,
                                 params->votes_min};
-        tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kBlock, msm, st>>>(a, tp, entropy, list, count);
+        tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kMaskThreads, msm, st>>>(a, tp, entropy, list, count);
+        const int rows = desc->B * desc->H * nkb;
+        tra::order_kernel<<<1, tra::kOrderThreads, (nkb + 1) * sizeof(int), st>>>(count, order, rows, nkb);
         return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
     }
     // block-sparse pass: the attention kernel walks the kept key blocks of the
@@ -732,6 +744,7 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
     a.kv_list = list;
     a.kv_count = count;
     a.kv_stride = nkb;
+    a.kv_order = order;
     return launch_tc(a, clean_pass, st) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
 }
 
@@ -774,9 +787,11 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
         return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
     }
     // bf16: the state chain (W_N = phi_q^T S_{N-1}, then S_N) on one stream, the
-    // attention kernels on another; attention of frame N waits only for W_N, so
-    // the attention kernels of consecutive frames share the SMs instead of each
-    // ending on a partial wave.  Each frame's W has its own slot.
+    // attention kernels on two others, frame after frame in turn; attention of
+    // frame N waits only for W_N, so the attention kernels of consecutive frames
+    // share the SMs (the next frame's first wave starts beside this frame's
+    // second) instead of each ending on a partial wave.  Each frame's W has its
+    // own slot.
     FrameRes* r = nullptr;
     if ((e = frame_resources(n_frames, &r)) != cudaSuccess) {
         delete[] args;
@@ -790,7 +805,15 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
         delete[] args;
         return HYB_ERR_INVALID;
     }
+    // the update runs beside attention kernels here, not in a partial wave of
+    // one: fewer CTAs per head (about a third of the SMs for all heads, at least
+    // two per head) cost less SM time for the same work
+    int fsplit = 0, ftokens = 0;
+    const int BH = desc->B * desc->H;
+    update_split(desc->T, kNumSMs / (3 * BH) > 2 ? kNumSMs / (3 * BH) : 2, true, &fsplit, &ftokens);
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
+        args[n].nsplit = fsplit;
+        args[n].split_tokens = ftokens;
         args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
         args[n].WT_lo = args[n].WT_hi + hh;
         // the update of frame n also writes W of frame n + 1 (what prep would
@@ -800,20 +823,22 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
     }
     if (e == cudaSuccess) e = cudaEventRecord(r->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(r->chain, r->fork, 0);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(r->att, r->fork, 0);
+    for (int i = 0; i < kAttStreams && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(r->att[i], r->fork, 0);
     if (e == cudaSuccess) e = tp[0].prep(r->chain, false);
     if (e == cudaSuccess) e = cudaEventRecord(r->w[0], r->chain);
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
         if ((e = tp[n].update(r->chain, false)) != cudaSuccess) break;
         if (n + 1 < n_frames && (e = cudaEventRecord(r->w[n + 1], r->chain)) != cudaSuccess) break;
-        if ((e = cudaStreamWaitEvent(r->att, r->w[n], 0)) != cudaSuccess) break;
-        e = tp[n].attn(r->att, false);
+        cudaStream_t att = r->att[n % kAttStreams];
+        if ((e = cudaStreamWaitEvent(att, r->w[n], 0)) != cudaSuccess) break;
+        e = tp[n].attn(att, false);
     }
     // join: the caller's stream continues after every frame's kernels
     if (e == cudaSuccess) e = cudaEventRecord(r->join_chain, r->chain);
-    if (e == cudaSuccess) e = cudaEventRecord(r->join_att, r->att);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, r->join_chain, 0);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, r->join_att, 0);
+    for (int i = 0; i < kAttStreams && e == cudaSuccess; ++i) {
+        if ((e = cudaEventRecord(r->join_att[i], r->att[i])) == cudaSuccess) e = cudaStreamWaitEvent(st, r->join_att[i], 0);
+    }
     delete[] tp;
     delete[] args;
     if (e == cudaSuccess) e = cudaGetLastError();

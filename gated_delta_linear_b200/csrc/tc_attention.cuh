@@ -129,7 +129,18 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     volatile int* epi_bad = (volatile int*)(tmem_slot + 2);  // a softmax warp missed its epilogue
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // the query tile of this CTA: its grid position, or the row that the
+    // schedule of a block-sparse pass gives it
+    int qt_ = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // (before a mask is built the schedule and the lengths are zero: grid order)
+    if (a.kv_order) {
+        const int row = a.kv_order[blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)];
+        if (a.kv_count[row] > 0) {
+            qt_ = row % gridDim.x;
+            h = (row / gridDim.x) % a.H;
+            b = row / (gridDim.x * a.H);
+        }
+    }
     const int T = a.T;
     const int q0 = qt_ * kTile;
     const int bh_ = b * a.H + h;

@@ -54,7 +54,9 @@ __host__ __device__ inline size_t mask_smem_bytes(int nkb) {
     return (size_t)nkb * (sizeof(int4) + 2 * sizeof(int) + kBlock * sizeof(int2));
 }
 
-// One CTA per (query block, head, batch), a thread per query of the block.
+// One CTA of kMaskThreads per (query block, head, batch): four warps per 32
+// queries of the block, each of the four taking every fourth key block (the
+// tests are short and latency-bound, so more warps per SM, not fewer, hide it).
 // Writes the ascending list of kept key blocks of the query block at
 // list[(bh * nkb + qb) * nkb] and its length at count[bh * nkb + qb].
 //
@@ -66,7 +68,9 @@ __host__ __device__ inline size_t mask_smem_bytes(int nkb) {
 // block fills its box (a whole tile, or rows of one), the box test alone is
 // exact.  Decisions are those of the per-key test: the same integer squared
 // distances against the same fp32 squared radius.
-__global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, const float* __restrict__ ent,
+constexpr int kMaskThreads = 512;
+constexpr int kKbGroups = kMaskThreads / kBlock;  // warps that share a query's key blocks
+__global__ void __launch_bounds__(kMaskThreads) mask_kernel(LayerArgs a, Params p, const float* __restrict__ ent,
                                                       int* __restrict__ list, int* __restrict__ count) {
     extern __shared__ __align__(16) unsigned char msm[];
     const int T = a.T;
@@ -78,9 +82,9 @@ __global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, con
     const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * a.H + h;
-    for (int kb = tid; kb < nkb; kb += kBlock) votes[kb] = 0;
+    for (int kb = tid; kb < nkb; kb += kMaskThreads) votes[kb] = 0;
     // runs and bounding box of each key block (a warp per block)
-    for (int kb = warp; kb < nkb; kb += kBlock / 32) {
+    for (int kb = warp; kb < nkb; kb += kMaskThreads / 32) {
         const int ntok = min(kBlock, T - kb * kBlock);
         int r0 = 1 << 30, r1 = -1, c0 = 1 << 30, c1 = -1;
         int nstart = 0, nend = 0;
@@ -120,12 +124,13 @@ __global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, con
         }
     }
     __syncthreads();
-    const int t = qb * kBlock + tid;
+    const int t = qb * kBlock + (warp % (kBlock / 32)) * 32 + lane;   // this thread's query
+    const int kb0 = warp / (kBlock / 32);                               // its first key block
     const bool valid = t < T;
     const float r2 = valid ? radius2(ent[bh * T + t], p.tau, T) : -1.0f;
     int rq = 0, cq = 0;
     if (valid) tile_major_pos(t, p, &rq, &cq);
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = kb0; kb < nkb; kb += kKbGroups) {
         const int4 bb = box[kb];
         const int dy = max(0, max(bb.x - rq, rq - bb.y)), dx = max(0, max(bb.z - cq, cq - bb.w));
         bool hit = false;
@@ -156,6 +161,33 @@ __global__ void __launch_bounds__(kBlock) mask_kernel(LayerArgs a, Params p, con
             if (votes[kb] >= p.votes_min || kb == qb) list[row * nkb + cnt++] = kb;
         count[row] = cnt;
     }
+}
+
+// The query-tile rows (bh * nkb + qb) ordered by the length of their key-block
+// lists, longest first (a counting sort; rows of equal length in any order, as
+// each row's result does not depend on when it runs).  The block-sparse
+// attention grid takes its rows in this order: CTAs are dispatched in grid
+// order, so the second wave holds the shortest rows and ends with the first.
+// One CTA; rows = B * H * nkb.
+constexpr int kOrderThreads = 1024;
+__global__ void __launch_bounds__(kOrderThreads) order_kernel(const int* __restrict__ count, int* __restrict__ order,
+                                                              int rows, int nkb) {
+    extern __shared__ int slot[];  // [nkb + 1]: rows of each length, then the first position of each length
+    for (int c = threadIdx.x; c <= nkb; c += kOrderThreads) slot[c] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < rows; i += kOrderThreads) atomicAdd(&slot[min(max(count[i], 0), nkb)], 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int pos = 0;
+        for (int c = nkb; c >= 0; --c) {
+            const int k = slot[c];
+            slot[c] = pos;
+            pos += k;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < rows; i += kOrderThreads)
+        order[atomicAdd(&slot[min(max(count[i], 0), nkb)], 1)] = i;
 }
 
 }  // namespace tra

@@ -133,3 +133,21 @@ def test_tra_huge_budget_is_the_dense_layer():
     assert G.hyb_attn_forward(desc, q, k, v, *phi, g, bl, S2, 1, o2, ws2) == G.HYB_OK
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_tra_sparse_pass_before_any_warmup_is_dense():
+    """No mask built on a fresh workspace: the block-sparse pass is the dense pass."""
+    import gated_delta_linear_b200 as G
+    w = W.small_workload(W.WORKLOADS[1], H=3, T=30 * 52, frames=1)
+    G_, params, desc, phi, ws, ent = _setup(w, 0.15, 2, (30, 52), (8, 16))
+    x = W.pass_inputs(w, 0, 0)
+    q, k, v, g, bl = (t.cuda() for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits))
+    S1 = torch.randn(w.B, w.H, w.d, w.d, dtype=torch.float32, device="cuda")
+    S2 = S1.clone()
+    o1 = torch.empty_like(q)
+    assert G.hyb_tra_forward(desc, params, 0, q, k, v, *phi, g, bl, S1, 1, o1, ent, ws) == G.HYB_OK
+    ws2 = torch.zeros(G.hyb_attn_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    o2 = torch.empty_like(q)
+    assert G.hyb_attn_forward(desc, q, k, v, *phi, g, bl, S2, 1, o2, ws2) == G.HYB_OK
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
