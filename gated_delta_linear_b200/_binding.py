@@ -86,8 +86,6 @@ def _load():
     L.hyb_attn_get_device_status.restype = i
     L.hyb_attn_set_fault_test.argtypes = [i, ctypes.c_uint]
     L.hyb_attn_set_fault_test.restype = i
-    L.hyb_attn_set_schedule_test.argtypes = [i]
-    L.hyb_attn_set_schedule_test.restype = i
     L.hyb_attn_timing_begin.argtypes = [i]
     L.hyb_attn_timing_begin.restype = i
     L.hyb_attn_timing_end.argtypes = [ctypes.POINTER(HybAttnTiming)]
@@ -236,11 +234,6 @@ def hyb_attn_set_fault_test(skip_v_loads: int, wait_limit_us: int) -> int:
     """Test hook (off by default): shorten the attention kernel's bounded waits
     and/or switch off its value-tile loads so that a wait expires."""
     return lib.hyb_attn_set_fault_test(int(skip_v_loads), int(wait_limit_us))
-
-
-def hyb_attn_set_schedule_test(mode: int) -> int:
-    """Test hook: which CTA of a split query tile merges (0 = normal)."""
-    return lib.hyb_attn_set_schedule_test(int(mode))
 
 
 def hyb_attn_timing_begin(max_launches: int) -> int:

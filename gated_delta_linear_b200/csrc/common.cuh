@@ -58,17 +58,9 @@ struct LayerArgs {
     // optional: CTA i of the grid takes query tile row kv_order[i] (bh * n_qt + qt),
     // so the longest lists go first
     const int* kv_order;
-    // the evenly divided attention grid: sk_grid CTAs (0: one CTA per query tile);
-    // partial records of rows split between two CTAs and their tickets
-    int sk_grid;
-    float* sk_part;
-    int* sk_cnt;
     // bounded device waits give up after wait_ns (2 s unless a fault test shortens it)
     unsigned long long wait_ns;
     int dbg_skip_v;            // fault test only: the attention kernel's V producer issues nothing
-    // schedule test only (evenly divided grid): 1 = tails take their ticket after their
-    // CTA's last item, 2 = heads do not look at the tail's ticket first
-    int dbg_sk_mode;
 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

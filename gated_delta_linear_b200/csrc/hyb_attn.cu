@@ -15,7 +15,6 @@
 #include "simt_layer.cuh"
 #include "tc_kernels.cuh"
 #include "tc_attention.cuh"
-#include "tc_attention_sk.cuh"
 #include "token_level.cuh"
 #include "tra.cuh"
 
@@ -30,7 +29,7 @@ struct Plan {
     bool bf16;
     int nsplit;
     int split_tokens;
-    size_t off_W, off_Sprev, off_part, off_sk, total;
+    size_t off_W, off_Sprev, off_part, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -45,22 +44,6 @@ void update_split(int T, int want, bool bf16, int* nsplit, int* split_tokens) {
     const int tiles_per_split = (ntiles + want - 1) / want;
     *split_tokens = tiles_per_split * kUpdateTile;
     *nsplit = (ntiles + tiles_per_split - 1) / tiles_per_split;
-}
-
-// One set of split-row records (two per boundary between consecutive CTAs of
-// the evenly divided attention grid) and their tickets.
-// (boundary c lies between CTAs c-1 and c, so 1 <= c < grid; one spare slot)
-size_t sk_rec_bytes() {
-    return align_up((size_t)(tc::sk::kMaxGrid + 1) * tc::sk::kSlotFloats * sizeof(float), 256);
-}
-size_t sk_set_bytes() { return sk_rec_bytes() + align_up((size_t)(tc::sk::kMaxGrid + 1) * sizeof(int), 256); }
-
-// CTAs of the evenly divided attention grid: one per SM, and at most one per
-// query tile (so that a CTA holds at least a whole row's units and a row is
-// split over at most two CTAs).
-int sk_grid(const hyb_attn_desc* d) {
-    const long long rows = (long long)d->B * d->H * ((d->T + 127) / 128);
-    return rows < kNumSMs ? (int)rows : kNumSMs;
 }
 
 hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
@@ -89,9 +72,7 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     p->off_part = align_up(p->off_Sprev + hh * sizeof(float), 256);
     // fp32 path: split partials (the tensor path reduces its splits on chip)
     const size_t part_bytes = bf16 ? 0 : hh * 2 * p->nsplit * sizeof(float);
-    // tensor path: records and tickets of the evenly divided attention grid
-    p->off_sk = align_up(p->off_part + part_bytes, 256);
-    p->total = p->off_sk + (bf16 ? sk_set_bytes() : 0);
+    p->total = align_up(p->off_part + part_bytes, 256);
     return HYB_OK;
 }
 
@@ -131,7 +112,6 @@ bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 struct FaultTest {
     int skip_v = 0;
     unsigned long long wait_ns = 2000000000ull;
-    int sk_mode = 0;  // schedule test: see hyb_attn_set_schedule_test in the header
 } g_fault;
 
 // Opt each kernel into its dynamic shared memory once per device.
@@ -267,8 +247,6 @@ struct TcPass {
         static unsigned char done_attn_ent[kMaxDevices];
         if ((e = opt_in_smem(tc::attention_kernel<false>, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
         if ((e = opt_in_smem(tc::attention_kernel<true>, tc::attn::SMEM, done_attn_ent)) != cudaSuccess) return e;
-        static unsigned char done_attn_sk[kMaxDevices];
-        if ((e = opt_in_smem(tc::attention_sk_kernel, tc::sk::SMEM, done_attn_sk)) != cudaSuccess) return e;
         if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
         const uint64_t row_bytes = (uint64_t)a.H * D * 2;
         const uint64_t bh = (uint64_t)a.B * a.H;
@@ -315,20 +293,10 @@ struct TcPass {
         cfg.attrs = at;
         cfg.numAttrs = pdl ? 1 : 0;
         cudaError_t le = cudaSuccess;
-        // a plain pass (bf16 output, O_inter = Q W): the evenly divided grid;
-        // otherwise one CTA per query tile (the entropy-writing variant for the
-        // warm-up pass of Token Radius Attention, block lists, branch outputs,
-        // the token-level read)
-        const bool even = a.sk_grid > 0 && a.sk_part && a.out && a.inter && !a.ent_out && !a.kv_count &&
-                          !a.oi_ext && !a.out_intra;
-        if (even) cfg.gridDim = dim3(a.sk_grid, 1, 1);
+        // the entropy-writing variant for the warm-up pass of Token Radius Attention
         cudaError_t e = timed(K_ATTN, st, [&] {
-            if (even)
-                le = cudaLaunchKernelEx(&cfg, tc::attention_sk_kernel, a, tq, tk, tv, tw, tout);
-            else if (a.ent_out)
-                le = cudaLaunchKernelEx(&cfg, tc::attention_kernel<true>, a, tq, tk, tv, tw, tout);
-            else
-                le = cudaLaunchKernelEx(&cfg, tc::attention_kernel<false>, a, tq, tk, tv, tw, tout);
+            le = a.ent_out ? cudaLaunchKernelEx(&cfg, tc::attention_kernel<true>, a, tq, tk, tv, tw, tout)
+                           : cudaLaunchKernelEx(&cfg, tc::attention_kernel<false>, a, tq, tk, tv, tw, tout);
         });
         return e != cudaSuccess ? e : le;
     }
@@ -426,14 +394,8 @@ hyb_status pass_args(const hyb_attn_desc* desc, const void* q, const void* k, co
     a.partials = (float*)(ws + p.off_part);
     a.nsplit = p.nsplit;
     a.split_tokens = p.split_tokens;
-    if (p.bf16) {
-        a.sk_grid = sk_grid(desc);
-        a.sk_part = (float*)(ws + p.off_sk);
-        a.sk_cnt = (int*)(ws + p.off_sk + sk_rec_bytes());
-    }
     a.wait_ns = g_fault.wait_ns;
     a.dbg_skip_v = g_fault.skip_v;
-    a.dbg_sk_mode = g_fault.sk_mode;
     *args = a;
     *plan = p;
     return HYB_OK;
@@ -582,11 +544,8 @@ size_t frames_w_bytes(const hyb_attn_desc* d, const Plan& p) {
     return (size_t)d->B * d->H * p.D * p.D * 2 * sizeof(__nv_bfloat16);
 }
 
-// bf16: the pass's workspace, one W per frame, and a second set of split-row
-// records for the attention kernels on the second attention stream
 size_t frames_total(const hyb_attn_desc* d, const Plan& p, int n) {
-    return align_up(p.total, 256) +
-           (p.bf16 ? (size_t)n * align_up(frames_w_bytes(d, p), 256) + sk_set_bytes() : 0);
+    return align_up(p.total, 256) + (p.bf16 ? (size_t)n * align_up(frames_w_bytes(d, p), 256) : 0);
 }
 
 hyb_status forward_impl(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
@@ -654,7 +613,6 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     a.flags = (unsigned*)workspace;
     a.wait_ns = g_fault.wait_ns;
     a.dbg_skip_v = g_fault.skip_v;
-    a.dbg_sk_mode = g_fault.sk_mode;
 
     static unsigned char done_attn[kMaxDevices];
     cudaError_t e;
@@ -853,14 +811,9 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
     int fsplit = 0, ftokens = 0;
     const int BH = desc->B * desc->H;
     update_split(desc->T, kNumSMs / (3 * BH) > 2 ? kNumSMs / (3 * BH) : 2, true, &fsplit, &ftokens);
-    char* sk2 = slots + n_frames * wslot;  // split-row records of the second attention stream
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
         args[n].nsplit = fsplit;
         args[n].split_tokens = ftokens;
-        if (n % kAttStreams == 1) {
-            args[n].sk_part = (float*)sk2;
-            args[n].sk_cnt = (int*)(sk2 + sk_rec_bytes());
-        }
         args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
         args[n].WT_lo = args[n].WT_hi + hh;
         // the update of frame n also writes W of frame n + 1 (what prep would
@@ -944,12 +897,6 @@ hyb_status hyb_attn_set_fault_test(int skip_v_loads, unsigned wait_limit_us) {
     if (wait_limit_us > 10u * 1000u * 1000u) return HYB_ERR_INVALID;
     g_fault.skip_v = skip_v_loads;
     g_fault.wait_ns = wait_limit_us ? (unsigned long long)wait_limit_us * 1000ull : 2000000000ull;
-    return HYB_OK;
-}
-
-hyb_status hyb_attn_set_schedule_test(int mode) {
-    if (mode < 0 || mode > 2) return HYB_ERR_INVALID;
-    g_fault.sk_mode = mode;
     return HYB_OK;
 }
 

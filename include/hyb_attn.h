@@ -311,19 +311,6 @@ hyb_status hyb_attn_get_device_status(const void* workspace, void* stream);
  * Not thread-safe; set it back to (0, 0) after the test. */
 hyb_status hyb_attn_set_fault_test(int skip_v_loads, unsigned wait_limit_us);
 
-/* ---- schedule test (tests only) -----------------------------------------------
- * Process-wide and off by default (mode 0); affects calls made after it.  The
- * plain pass's attention grid may split a 128-query tile between two CTAs: the
- * head (its first key tiles) and the tail (its last).  The one whose ticket
- * comes second merges the two partial softmax sums, and which one that is
- * depends on timing.  mode 1: tails take their ticket only after the rest of
- * their CTA's work, so heads publish and tails merge from the two records.
- * mode 2: heads do not look at the tail's ticket before taking their own, so
- * they publish and, when second, merge from global memory instead of shared
- * memory.  The results are bit-identical to mode 0's.  HYB_ERR_INVALID for a
- * mode outside {0, 1, 2}.  Not thread-safe; set it back to 0 after the test. */
-hyb_status hyb_attn_set_schedule_test(int mode);
-
 /* ---- optional kernel timing (benchmarks) ------------------------------------
  * Process-wide and off by default.  hyb_attn_timing_begin(n) creates 2n CUDA
  * events on the current device; until hyb_attn_timing_end, every kernel that

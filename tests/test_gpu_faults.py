@@ -18,13 +18,6 @@ import workloads as W
 from tests import tolerances as tol
 
 
-def test_schedule_test_knob_validates_its_argument():
-    import gated_delta_linear_b200 as G
-    assert G.hyb_attn_set_schedule_test(3) == G.HYB_ERR_INVALID
-    assert G.hyb_attn_set_schedule_test(-1) == G.HYB_ERR_INVALID
-    assert G.hyb_attn_set_schedule_test(0) == G.HYB_OK
-
-
 def test_fault_test_knob_validates_its_arguments():
     import gated_delta_linear_b200 as G
     assert G.hyb_attn_set_fault_test(2, 0) == G.HYB_ERR_INVALID

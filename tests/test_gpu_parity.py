@@ -138,11 +138,6 @@ def test_query_only_pass_leaves_state_bit_identical():
 
 
 def test_forward_equals_branches_and_is_deterministic():
-    """The plain pass runs the evenly divided attention grid, the branch entry
-    point one CTA per query tile: the same arithmetic except where a query tile
-    is split between two CTAs and its two partial softmax sums are merged, so
-    outputs agree to one bf16 step and the states (the same update kernel) bit
-    for bit; the plain pass is deterministic."""
     w = W.small_workload(W.WORKLOADS[1], frames=3)
     outs = []
     for mode in ("forward", "branches", "forward"):
@@ -156,11 +151,8 @@ def test_forward_equals_branches_and_is_deterministic():
                 o, oi, oe = L.forward_branches(q, k, v, g, bl, True)
         torch.cuda.synchronize()
         outs.append((o.clone(), L.state.clone()))
-    assert torch.equal(outs[2][0], outs[0][0]) and torch.equal(outs[2][1], outs[0][1])
-    assert torch.equal(outs[1][1], outs[0][1])
-    a, b = outs[0][0].float(), outs[1][0].float()
-    step = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 1e-6 * a.abs().max().item()
-    assert bool(((a - b).abs() <= step).all())
+    for o, s in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
 
 
 def test_checkpoint_resume_bit_identical():
@@ -210,38 +202,3 @@ def test_device_side_argument_errors():
     st = G.hyb_attn_forward(L.desc, qq.data_ptr() + 2, k, v, *L.phi, g, bl, L.state, 1, out,
                             L.workspace)
     assert st == G.HYB_ERR_ALIGN
-
-
-@pytest.mark.gpu
-def test_split_tile_merges_agree_in_every_schedule():
-    """The plain pass splits query tiles between two CTAs (480p: 156 tiles on 148
-    CTAs); whichever CTA merges, and from wherever it reads the other's partial
-    sums, the outputs are bit-identical, and they match the oracle."""
-    import gated_delta_linear_b200 as G
-    import oracle
-    w = W.small_workload(W.WORKLOADS[1], frames=2)
-    runs = []
-    try:
-        for mode in (0, 1, 2):
-            assert G.hyb_attn_set_schedule_test(mode) == G.HYB_OK
-            L = _layer(w)
-            outs = []
-            for n in range(w.frames):
-                outs.append(L.forward(*_dev_inputs(w, n, 0), True).clone())
-            torch.cuda.synchronize()
-            assert L.device_status() == G.HYB_OK
-            runs.append((outs, L.state.clone()))
-    finally:
-        G.hyb_attn_set_schedule_test(0)
-    for outs, st in runs[1:]:
-        assert torch.equal(st, runs[0][1])
-        for a, b in zip(outs, runs[0][0]):
-            assert torch.equal(a, b)
-    phi64 = [p.double().numpy() for p in W.feature_maps(w)]
-    S = W.zero_state(w)
-    for n in range(w.frames):
-        x = W.pass_inputs(w, n, 0)
-        ref, _, _, S = oracle.layer_pass(*x.as_f64()[:3], *phi64, *x.as_f64()[3:], S, True)
-        got = runs[1][0][n].double().cpu().numpy()
-        for h in range(w.H):
-            tol.check(tol.scaled_errors(got[0, :, h], ref[0, :, h]), tol.OUT_BF16, f"frame {n} head {h}")

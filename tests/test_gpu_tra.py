@@ -57,14 +57,11 @@ def _run(w, tau, votes_min, grid, tiles, frames=2):
         x = W.pass_inputs(w, n, 0)
         q, k, v, g, bl = (t.cuda() for t in (x.q, x.k, x.v, x.gate_logits, x.beta_logits))
         q64, k64, v64, g64, bl64 = x.as_f64()
-        # warm-up: the dense pass plus entropies, bit-identical to the one-CTA-per-tile
-        # dense pass (the branch entry point runs that kernel)
+        # warm-up: the dense pass, bit-identical to hyb_attn_forward, plus entropies
         ws_ref = torch.zeros(G.hyb_attn_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
         S_chk = S_gpu.clone()
         o_ref = torch.empty_like(q)
-        f32 = lambda: torch.empty(q.shape, dtype=torch.float32, device="cuda")
-        assert G.hyb_attn_forward_branches(desc, q, k, v, *phi, g, bl, S_chk, 0, o_ref, f32(), f32(),
-                                           ws_ref) == G.HYB_OK
+        assert G.hyb_attn_forward(desc, q, k, v, *phi, g, bl, S_chk, 0, o_ref, ws_ref) == G.HYB_OK
         o_w = torch.empty_like(q)
         assert G.hyb_tra_forward(desc, params, 1, q, k, v, *phi, g, bl, S_gpu, 0, o_w, ent, ws) == G.HYB_OK
         torch.cuda.synchronize()
