@@ -465,26 +465,52 @@ def run_cuda(args):
     h2d = sum(t.numel() * t.element_size() for f in pin for t in f)
     d2h = sum(o.numel() * o.element_size() for o in hout)
 
+    # The step as a user streaming video would run it: the inputs arrive in
+    # pieces (chunks of frames for the frames call, else one pass at a time);
+    # a copy stream brings each piece in, the compute stream runs it once it has
+    # arrived, and a second copy stream takes its outputs back, so copies in
+    # both directions overlap each other and the compute.
+    if frames_api:
+        cf = 7
+        units = []
+        for k0 in range(0, len(host), cf):
+            k1 = min(len(host), k0 + cf)
+            call = [dref, k1 - k0] + [stk[i][k0].data_ptr() for i in range(3)] + phis + \
+                   [stk[3][k0].data_ptr(), stk[4][k0].data_ptr(), state_ptr, out_stk[k0].data_ptr(),
+                    fws.data_ptr(), fws.numel(), sptr]
+            units.append((list(range(k0, k1)), call))
+    else:
+        units = [([n], None) for n in range(len(host))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in units]
+    ev_comp = [torch.cuda.Event() for _ in units]
+    ev_out = [torch.cuda.Event() for _ in units]
+
     def e2e_step():
         layer.state.copy_(state0)
-        if frames_api:
-            # every frame's inputs in, one call, every frame's output back
-            for f, hf in zip(frames, pin):
-                for dst, src_ in zip(f, hf):
-                    dst.copy_(src_, non_blocking=True)
-            st = G.lib.hyb_attn_forward_frames(*fcall)
-            if st != G.HYB_OK:
-                raise G.HybAttnError(st, "hyb_attn_forward_frames")
-            for o, ho in zip(outs, hout):
-                ho.copy_(o, non_blocking=True)
-            return
-        for f, hf, c, o, ho in zip(frames, pin, calls, outs, hout):
-            for dst, src_ in zip(f, hf):
-                dst.copy_(src_, non_blocking=True)
-            st = fwd(dref, *c)
-            if st != G.HYB_OK:
-                raise G.HybAttnError(st, "hyb_attn_forward")
-            ho.copy_(o, non_blocking=True)
+        for u, (idx, call) in enumerate(units):
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[u])          # the previous step has read these inputs
+                for n in idx:
+                    for dst, src_ in zip(frames[n], pin[n]):
+                        dst.copy_(src_, non_blocking=True)
+                ev_in[u].record(s_in)
+            stream.wait_event(ev_in[u])
+            stream.wait_event(ev_out[u])             # the previous step's outputs are out
+            if call is not None:
+                st = G.lib.hyb_attn_forward_frames(*call)
+                if st != G.HYB_OK:
+                    raise G.HybAttnError(st, "hyb_attn_forward_frames")
+            else:
+                st = fwd(dref, *calls[idx[0]])
+                if st != G.HYB_OK:
+                    raise G.HybAttnError(st, "hyb_attn_forward")
+            ev_comp[u].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[u])
+                for n in idx:
+                    hout[n].copy_(outs[n], non_blocking=True)
+                ev_out[u].record(s_out)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -492,8 +518,10 @@ def run_cuda(args):
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_in.wait_stream(stream)
     for _ in range(e2e_steps):
         e2e_step()
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
@@ -525,7 +553,11 @@ def run_cuda(args):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "schedule": ("inputs in chunks of 7 frames on a copy stream, one frames call per chunk "
+                             "once it has arrived, outputs back on a second copy stream")
+                if frames_api else ("one pass at a time: inputs on a copy stream, the pass once they "
+                                    "have arrived, outputs back on a second copy stream")},
         "api": ("hyb_attn_forward_frames (one call per 21-frame forward: the kernels of one "
                 "hyb_attn_forward call per frame, scheduled over three streams)") if frames_api else "hyb_attn_forward (one call per pass)",
         "per_frame_calls": {"value": job_throughput(tokens_per_step, args.steps, world, ms_loop), "unit": UNIT,
