@@ -45,6 +45,7 @@ from ._binding import (  # noqa: F401
     HybAttnTiming,
     HYB_NUM_KERNELS,
     hyb_attn_set_fault_test,
+    hyb_attn_noalloc_device_status,
     hyb_attn_timing_begin,
     hyb_attn_timing_end,
     hyb_attn_kernel_name,

@@ -86,6 +86,8 @@ def _load():
     L.hyb_attn_get_device_status.restype = i
     L.hyb_attn_set_fault_test.argtypes = [i, ctypes.c_uint]
     L.hyb_attn_set_fault_test.restype = i
+    L.hyb_attn_noalloc_device_status.argtypes = [vp]
+    L.hyb_attn_noalloc_device_status.restype = i
     L.hyb_attn_timing_begin.argtypes = [i]
     L.hyb_attn_timing_begin.restype = i
     L.hyb_attn_timing_end.argtypes = [ctypes.POINTER(HybAttnTiming)]
@@ -228,6 +230,11 @@ def hyb_attn_get_device_status(workspace, stream=None) -> int:
 
 def hyb_attn_status_string(status: int) -> str:
     return lib.hyb_attn_status_string(int(status)).decode()
+
+
+def hyb_attn_noalloc_device_status(stream=None) -> int:
+    """Status flags of the last hyb_attn_forward_noalloc call on the current device."""
+    return lib.hyb_attn_noalloc_device_status(_stream(stream))
 
 
 def hyb_attn_set_fault_test(skip_v_loads: int, wait_limit_us: int) -> int:

@@ -1033,3 +1033,11 @@ extern "C" hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc, const 
         return HYB_ERR_CUDA;
     return launch_pass(a, p, clean_pass, stream);
 }
+
+extern "C" hyb_status hyb_attn_noalloc_device_status(void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYB_ERR_CUDA;
+    // the scratch address is known once a call on this device has looked it up
+    if (!g_noalloc_ptr[dev]) return HYB_OK;
+    return hyb_attn_get_device_status(g_noalloc_ptr[dev], stream);
+}

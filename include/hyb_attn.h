@@ -188,13 +188,20 @@ hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc,
  * and it keeps the last call's contents: calls that can overlap on the GPU
  * (different streams, concurrent threads) race on it and must be serialised by
  * the caller.  Device status flags of these calls are cleared at the start of
- * each call and are not reported by hyb_attn_get_device_status. */
+ * each call; hyb_attn_noalloc_device_status reports those of the last call. */
 #define HYB_NOALLOC_SCRATCH_BYTES (32u << 20)
 hyb_status hyb_attn_forward_noalloc(const hyb_attn_desc* desc,
                                     const void* q, const void* k, const void* v,
                                     const void* phi_q, const void* phi_k, const void* phi_v,
                                     const float* gate_logits, const float* beta_logits,
                                     float* state, int clean_pass, void* out, void* stream);
+
+/* hyb_attn_noalloc_device_status -- synchronises `stream`, then reads and
+ * clears the device status flags of the last hyb_attn_forward_noalloc call on
+ * the current device (in the library's scratch array), with the meaning of
+ * hyb_attn_get_device_status.  HYB_OK if no such call was made on this device.
+ * Allocates nothing. */
+hyb_status hyb_attn_noalloc_device_status(void* stream);
 
 /* hyb_attn_forward_token_level -- the token-level access variant of a pass
  * (ARL2 summary §4, ablations: token-level against frame-level access to the

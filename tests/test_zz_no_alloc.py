@@ -94,3 +94,27 @@ def test_noalloc_rejects_bad_arguments_before_any_cuda_call(what):
         want = G.HYB_ERR_INVALID
     assert G.hyb_attn_forward_noalloc(desc, *args, 0) == want
 
+
+
+@pytest.mark.gpu
+def test_noalloc_status_getter_reports_the_last_call():
+    """The no-allocation entry point's device flags: HYB_OK after a normal call;
+    after a call whose bounded wait is made to run out (the fault test), the
+    getter reports HYB_ERR_TIMEOUT, and a normal call afterwards is HYB_OK again."""
+    import gated_delta_linear_b200 as G
+    w = W.small_workload(W.WORKLOADS[1], H=2, T=300, frames=1)
+    phi = [p.cuda() for p in W.feature_maps(w)]
+    desc = G.make_desc(w.B, w.H, w.T, w.d, G.HYB_BF16)
+    q, k, v, g, bl = _inputs(w, 0, 0)
+    S = torch.zeros(w.B, w.H, w.d, w.d, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(q)
+    assert G.hyb_attn_forward_noalloc(desc, q, k, v, *phi, g, bl, S, 0, out) == G.HYB_OK
+    assert G.hyb_attn_noalloc_device_status() == G.HYB_OK
+    assert G.hyb_attn_set_fault_test(1, 5000) == G.HYB_OK
+    try:
+        assert G.hyb_attn_forward_noalloc(desc, q, k, v, *phi, g, bl, S, 0, out) == G.HYB_OK
+        assert G.hyb_attn_noalloc_device_status() == G.HYB_ERR_TIMEOUT
+    finally:
+        G.hyb_attn_set_fault_test(0, 0)
+    assert G.hyb_attn_forward_noalloc(desc, q, k, v, *phi, g, bl, S, 0, out) == G.HYB_OK
+    assert G.hyb_attn_noalloc_device_status() == G.HYB_OK
