@@ -558,8 +558,8 @@ def run_cuda(args):
                              "once it has arrived, outputs back on a second copy stream")
                 if frames_api else ("one pass at a time: inputs on a copy stream, the pass once they "
                                     "have arrived, outputs back on a second copy stream")},
-        "api": ("hyb_attn_forward_frames (one call per 21-frame forward: the kernels of one "
-                "hyb_attn_forward call per frame, scheduled over three streams)") if frames_api else "hyb_attn_forward (one call per pass)",
+        "api": ("hyb_attn_forward_frames (one call per 21-frame forward, bit-identical to one "
+                "hyb_attn_forward call per frame)") if frames_api else "hyb_attn_forward (one call per pass)",
         "per_frame_calls": {"value": job_throughput(tokens_per_step, args.steps, world, ms_loop), "unit": UNIT,
                             "us_per_frame": 1e3 * ms_loop / args.steps / w.frames,
                             "api": "hyb_attn_forward, one call per pass (the autoregressive pattern)"},

@@ -62,10 +62,15 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     p->bf16 = bf16;
     // token splits of the state update, each a whole number of 128-token tiles.
     // Tensor path: one cluster of at most 8 CTAs per (b, h), splits reduced in
-    // distributed shared memory (no partials in the workspace).  fp32 path:
-    // enough (b, h, split) blocks to cover the SMs, partials in the workspace.
+    // distributed shared memory (no partials in the workspace).  The update runs
+    // beside attention kernels (the second wave of its own frame's, or the next
+    // frame's), so its splits take about a third of the SMs in all and at least 3
+    // per head: fewer CTAs per head cost less SM time for the same work, more
+    // shorten the chain from one frame's state to the next.  fp32 path: enough
+    // (b, h, split) blocks to cover the SMs, partials in the workspace.
     const int BH = d->B * d->H;
-    update_split(d->T, bf16 ? kNumSMs / BH : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
+    const int third = kNumSMs / (3 * BH) > 3 ? kNumSMs / (3 * BH) : 3;
+    update_split(d->T, bf16 ? third : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
     const size_t hh = (size_t)BH * D * D;
     p->off_W = kStatusBytes;
     p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
@@ -805,15 +810,7 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
         delete[] args;
         return HYB_ERR_INVALID;
     }
-    // the update runs beside attention kernels here, not in a partial wave of
-    // one: fewer CTAs per head (about a third of the SMs for all heads, at least
-    // two per head) cost less SM time for the same work
-    int fsplit = 0, ftokens = 0;
-    const int BH = desc->B * desc->H;
-    update_split(desc->T, kNumSMs / (3 * BH) > 2 ? kNumSMs / (3 * BH) : 2, true, &fsplit, &ftokens);
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
-        args[n].nsplit = fsplit;
-        args[n].split_tokens = ftokens;
         args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
         args[n].WT_lo = args[n].WT_hi + hh;
         // the update of frame n also writes W of frame n + 1 (what prep would

@@ -121,13 +121,9 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
  * S_N, frame after frame) on one internal stream and the attention kernels on
  * two others, frame after frame in turn, each attention kernel waiting only for
  * its own W_N: the attention kernels of consecutive frames share the SMs.  The
- * kernels are those of the loop; the state update is split over fewer CTAs per
- * head (about a third of the SMs in all, since here it runs beside attention
- * kernels instead of filling a partial wave), so the state's sums are grouped
- * differently: the results agree with the loop to fp32 rounding of the state
- * (and the bf16 rounding of outputs that follows), not bit for bit.  For the
- * fp32 path the call is the loop.  The internal streams (the chain's at the
- * highest priority) and events
+ * results are bit-identical to the loop: the same kernels with the same
+ * arithmetic; only their scheduling differs (for the fp32 path the call is the
+ * loop).  The internal streams (the chain's at the highest priority) and events
  * are created on the first call on a device and kept; the call forks from and
  * joins back to `stream`, so work enqueued on `stream` afterwards sees every
  * output and the final state.  Not thread-safe.
