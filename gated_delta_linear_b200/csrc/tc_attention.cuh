@@ -250,6 +250,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
+            // descriptors of the first K stage (K-major and, for W, MN-major) and of
+            // the first V stage; a stage's descriptor is this plus its offset / 16
+            const uint64_t dK = kmajor_desc(sb + K0, 0), dW = mnmajor_desc(sb + K0, 0), dV = mnmajor_desc(sb + V0, 0);
+            constexpr uint64_t kStage = kTileBytes >> 4;
             // S_0 and S_1 take Q from shared memory (no wait for its copy into TMEM)
             bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns);
             bool q_in_tmem = false;
@@ -271,10 +275,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags, a.wait_ns))) break;
                     if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags, a.wait_ns))) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tS0 + sbuf * 128, tQ + kk * 8, kmajor_desc(sb + K0 + ks * kTileBytes, kk), ID_KK,
-                                    kk > 0);
+                    mma8_ts<false>(tS0 + sbuf * 128, tQ, dK + ks * kStage, ID_KK, 0);
                     mma_commit(&bars[B_SFULL + sbuf]);
                     mma_commit(&bars[B_KEMPTY + ks]);
                 }
@@ -288,21 +289,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                         break;
                     if (!(ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags, a.wait_ns))) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_hi * kTileBytes, kk), ID_KMN, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tOI, tQ + kk * 8, mnmajor_desc(sb + K0 + wst_lo * kTileBytes, kk), ID_KMN, 1);
+                    mma8_ts<true>(tOI, tQ, dW + wst_hi * kStage, ID_KMN, 0);
+                    mma8_ts<true>(tOI, tQ, dW + wst_lo * kStage, ID_KMN, 1);
                     mma_commit(&bars[B_OIDONE]);
                 }
                 const int vs = j % kVStages;
                 if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags, a.wait_ns))) break;
                 if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags, a.wait_ns))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tO, tP + kk * 8, mnmajor_desc(sb + V0 + vs * kTileBytes, kk), ID_KMN, (j > 0 || kk > 0));
+                mma8_ts<true>(tO, tP, dV + vs * kStage, ID_KMN, j > 0);
                 mma_commit(&bars[B_PVDONE]);
                 mma_commit(&bars[B_VEMPTY + vs]);
             }

@@ -42,6 +42,24 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     return sdesc_sw128(base + kk * 2048, kHalf, 1024);
 }
 
+// A descriptor's start-address field is its low 14 bits (the shared-memory
+// address / 16, all addresses below 256 KB), so the descriptor of slice kk is
+// the tile's descriptor (slice 0) plus a constant; the MMA issuing thread then
+// spends one add per MMA on its operands.
+__device__ __forceinline__ uint64_t kmajor_step(int kk) { return (uint64_t)((kk >> 2) * (kHalf >> 4) + (kk & 3) * 2); }
+__device__ __forceinline__ uint64_t mnmajor_step(int kk) { return (uint64_t)(kk * (2048 >> 4)); }
+
+// Eight MMAs D (+)= A_kk B_kk over the K slices kk = 0..7 of one 128-deep
+// product, A in TMEM (columns a_tmem + 8 kk), B from shared-memory descriptors
+// b0 + step(kk); the first accumulates into D if acc0, the rest always.
+template <bool kMnB>
+__device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc, uint32_t acc0) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ts(d_tmem, a_tmem + kk * 8, b0 + (kMnB ? mnmajor_step(kk) : kmajor_step(kk)), idesc,
+                    kk > 0 ? 1u : acc0);
+}
+
 // Max of N scores (fmaxf: NaN entries are skipped).
 template <int N>
 __device__ __forceinline__ float row_max(const float* x) {
