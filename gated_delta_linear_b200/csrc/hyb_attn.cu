@@ -700,9 +700,10 @@ size_t hyb_tra_workspace_bytes(const hyb_attn_desc* desc) {
     if (make_plan(desc, &p) != HYB_OK || !p.bf16) return 0;
     const size_t nkb = (desc->T + tra::kBlock - 1) / tra::kBlock;
     const size_t bh = (size_t)desc->B * desc->H;
-    // block lists, their lengths, the schedule of the block-sparse grid
+    // block lists, their lengths, the schedule of the block-sparse grid, the mask
+    // kernel's ticket
     return align_up(align_up(p.total, 256) + bh * nkb * nkb * sizeof(int), 256) +
-           2 * align_up(bh * nkb * sizeof(int), 256);
+           2 * align_up(bh * nkb * sizeof(int), 256) + 256;
 }
 
 hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* params, int warmup, const void* q,
@@ -727,6 +728,7 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
     int* list = (int*)((char*)workspace + align_up(p.total, 256));
     int* count = (int*)((char*)list + align_up((size_t)desc->B * desc->H * nkb * nkb * sizeof(int), 256));
     int* order = (int*)((char*)count + align_up((size_t)desc->B * desc->H * nkb * sizeof(int), 256));
+    int* done = (int*)((char*)order + align_up((size_t)desc->B * desc->H * nkb * sizeof(int), 256));
     const size_t msm = tra::mask_smem_bytes(nkb);
     if (msm > 227u * 1024u) return HYB_ERR_UNSUPPORTED;
     if (warmup) {
@@ -739,9 +741,8 @@ hyb_status hyb_tra_forward(const hyb_attn_desc* desc, const hyb_tra_params* para
         if (launch_tc(a, clean_pass, st) != cudaSuccess) return HYB_ERR_CUDA;
         const tra::Params tp = {params->grid_h, params->grid_w, params->tile_h, params->tile_w, params->tau,
                                 params->votes_min};
-        tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kMaskThreads, msm, st>>>(a, tp, entropy, list, count);
-        const int rows = desc->B * desc->H * nkb;
-        tra::order_kernel<<<1, tra::kOrderThreads, (nkb + 1) * sizeof(int), st>>>(count, order, rows, nkb);
+        tra::mask_kernel<<<dim3(nkb, desc->H, desc->B), tra::kMaskThreads, msm, st>>>(a, tp, entropy, list, count,
+                                                                                       order, done);
         return cudaGetLastError() == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
     }
     // block-sparse pass: the attention kernel walks the kept key blocks of the

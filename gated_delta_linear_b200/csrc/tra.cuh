@@ -58,7 +58,13 @@ __host__ __device__ inline size_t mask_smem_bytes(int nkb) {
 // queries of the block, each of the four taking every fourth key block (the
 // tests are short and latency-bound, so more warps per SM, not fewer, hide it).
 // Writes the ascending list of kept key blocks of the query block at
-// list[(bh * nkb + qb) * nkb] and its length at count[bh * nkb + qb].
+// list[(bh * nkb + qb) * nkb] and its length at count[bh * nkb + qb].  The CTA
+// that finishes last (an atomic ticket on *done, which it resets) then orders
+// the rows (bh * nkb + qb) by list length, longest first, into order[]: a
+// counting sort (rows of equal length in any order, as each row's result does
+// not depend on when it runs).  The block-sparse attention grid takes its rows
+// in this order: CTAs are dispatched in grid order, so its second wave holds
+// the shortest lists and ends with the first.
 //
 // A key block is described by its bounding box and by its runs: maximal
 // stretches of consecutive tokens on one patch row with consecutive columns
@@ -71,7 +77,8 @@ __host__ __device__ inline size_t mask_smem_bytes(int nkb) {
 constexpr int kMaskThreads = 512;
 constexpr int kKbGroups = kMaskThreads / kBlock;  // warps that share a query's key blocks
 __global__ void __launch_bounds__(kMaskThreads) mask_kernel(LayerArgs a, Params p, const float* __restrict__ ent,
-                                                      int* __restrict__ list, int* __restrict__ count) {
+                                                      int* __restrict__ list, int* __restrict__ count,
+                                                      int* __restrict__ order, int* __restrict__ done) {
     extern __shared__ __align__(16) unsigned char msm[];
     const int T = a.T;
     const int nkb = (T + kBlock - 1) / kBlock;
@@ -154,30 +161,33 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(LayerArgs a, Params 
         if (lane == 0 && nv) atomicAdd(&votes[kb], nv);
     }
     __syncthreads();
+    volatile int* last = nrun;  // (free now) the ticket's verdict for the whole CTA
     if (tid == 0) {
         const size_t row = bh * nkb + qb;
         int cnt = 0;
         for (int kb = 0; kb < nkb; ++kb)
             if (votes[kb] >= p.votes_min || kb == qb) list[row * nkb + cnt++] = kb;
         count[row] = cnt;
+        __threadfence();
+        const int ctas = gridDim.x * gridDim.y * gridDim.z;
+        const int ticket = atomicAdd(done, 1);
+        *last = ticket == ctas - 1;
+        if (ticket == ctas - 1) {
+            *done = 0;  // for the next mask
+            __threadfence();
+        }
     }
-}
-
-// The query-tile rows (bh * nkb + qb) ordered by the length of their key-block
-// lists, longest first (a counting sort; rows of equal length in any order, as
-// each row's result does not depend on when it runs).  The block-sparse
-// attention grid takes its rows in this order: CTAs are dispatched in grid
-// order, so the second wave holds the shortest rows and ends with the first.
-// One CTA; rows = B * H * nkb.
-constexpr int kOrderThreads = 1024;
-__global__ void __launch_bounds__(kOrderThreads) order_kernel(const int* __restrict__ count, int* __restrict__ order,
-                                                              int rows, int nkb) {
-    extern __shared__ int slot[];  // [nkb + 1]: rows of each length, then the first position of each length
-    for (int c = threadIdx.x; c <= nkb; c += kOrderThreads) slot[c] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < rows; i += kOrderThreads) atomicAdd(&slot[min(max(count[i], 0), nkb)], 1);
+    if (!*last) return;
+    // the last CTA: counting sort of the rows by list length (every CTA's count
+    // is visible: each wrote it before its ticket)
+    const int rows = gridDim.x * gridDim.y * gridDim.z;
+    int* slot = reinterpret_cast<int*>(box);  // [nkb + 1]: rows of each length, then first positions
+    for (int c = tid; c <= nkb; c += kMaskThreads) slot[c] = 0;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    for (int i = tid; i < rows; i += kMaskThreads) atomicAdd(&slot[min(max(__ldcg(count + i), 0), nkb)], 1);
+    __syncthreads();
+    if (tid == 0) {
         int pos = 0;
         for (int c = nkb; c >= 0; --c) {
             const int k = slot[c];
@@ -186,8 +196,8 @@ __global__ void __launch_bounds__(kOrderThreads) order_kernel(const int* __restr
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < rows; i += kOrderThreads)
-        order[atomicAdd(&slot[min(max(count[i], 0), nkb)], 1)] = i;
+    for (int i = tid; i < rows; i += kMaskThreads)
+        order[atomicAdd(&slot[min(max(__ldcg(count + i), 0), nkb)], 1)] = i;
 }
 
 }  // namespace tra
