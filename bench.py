@@ -353,6 +353,19 @@ def run_cuda(args):
             if st != G.HYB_OK:
                 raise G.HybAttnError(st, "hyb_attn_forward")
 
+    # one call per pass through hyb_attn_forward_next: the restored state starts
+    # a new chain (a plain pass), every later pass continues it (the W of the
+    # next frame comes from the previous clean pass's update, and each attention
+    # kernel starts while the previous update still runs)
+    fwd_next = G.lib.hyb_attn_forward_next
+
+    def step_next():
+        layer.state.copy_(state0)
+        for i, c in enumerate(calls):
+            st = (fwd if i == 0 else fwd_next)(dref, *c)
+            if st != G.HYB_OK:
+                raise G.HybAttnError(st, "hyb_attn_forward_next")
+
     if frames_api:
         nf = len(host)
         fws = torch.zeros(G.hyb_attn_frames_workspace_bytes(desc, nf), dtype=torch.uint8, device=dev)
@@ -365,7 +378,7 @@ def run_cuda(args):
             if st != G.HYB_OK:
                 raise G.HybAttnError(st, "hyb_attn_forward_frames")
     else:
-        step = step_loop
+        step = step_next
 
     if args.profile_run:
         # kernel order per frame: prep, intra_frame_attention, delta_update
@@ -378,6 +391,8 @@ def run_cuda(args):
     for _ in range(max(3, args.warmup)):
         step()
         step_loop()
+        if frames_api:
+            step_next()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -393,18 +408,21 @@ def run_cuda(args):
         stop.record(stream)
         torch.cuda.synchronize(dev)
     ms = max_over_ranks(start.elapsed_time(stop), dev)
-    # the same steps as one hyb_attn_forward call per pass (autoregressive use:
-    # the next frame's inputs exist only after this frame)
-    ms_loop = ms
-    if frames_api:
+    # the same steps as one call per pass (autoregressive use: the next frame's
+    # inputs exist only after this frame), through hyb_attn_forward and through
+    # hyb_attn_forward_next
+    def time_steps(fn):
         if world > 1:
             dist.barrier()
         start.record(stream)
         for _ in range(args.steps):
-            step_loop()
+            fn()
         stop.record(stream)
         torch.cuda.synchronize(dev)
-        ms_loop = max_over_ranks(start.elapsed_time(stop), dev)
+        return max_over_ranks(start.elapsed_time(stop), dev)
+
+    ms_loop = time_steps(step_loop)
+    ms_next = time_steps(step_next) if frames_api else ms
     # timed region B: the per-pass calls with the library's timing hook, which
     # brackets every kernel with events on the library's stream (per-kernel durations)
     n_launch_cap = args.steps * w.frames * len(w.passes) * G.HYB_NUM_KERNELS + 16
@@ -502,9 +520,9 @@ def run_cuda(args):
                 if st != G.HYB_OK:
                     raise G.HybAttnError(st, "hyb_attn_forward_frames")
             else:
-                st = fwd(dref, *calls[idx[0]])
+                st = (fwd if idx[0] == 0 else fwd_next)(dref, *calls[idx[0]])
                 if st != G.HYB_OK:
-                    raise G.HybAttnError(st, "hyb_attn_forward")
+                    raise G.HybAttnError(st, "hyb_attn_forward_next")
             ev_comp[u].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[u])
@@ -557,12 +575,19 @@ def run_cuda(args):
                 "schedule": ("inputs in chunks of 7 frames on a copy stream, one frames call per chunk "
                              "once it has arrived, outputs back on a second copy stream")
                 if frames_api else ("one pass at a time: inputs on a copy stream, the pass once they "
-                                    "have arrived, outputs back on a second copy stream")},
+                                    "have arrived (hyb_attn_forward_next), outputs back on a second "
+                                    "copy stream")},
         "api": ("hyb_attn_forward_frames (one call per 21-frame forward, bit-identical to one "
-                "hyb_attn_forward call per frame)") if frames_api else "hyb_attn_forward (one call per pass)",
+                "hyb_attn_forward call per frame)") if frames_api else
+               ("hyb_attn_forward_next (one call per pass; the first pass of a step, on the restored "
+                "state, through hyb_attn_forward; bit-identical to hyb_attn_forward per pass)"),
         "per_frame_calls": {"value": job_throughput(tokens_per_step, args.steps, world, ms_loop), "unit": UNIT,
                             "us_per_frame": 1e3 * ms_loop / args.steps / w.frames,
                             "api": "hyb_attn_forward, one call per pass (the autoregressive pattern)"},
+        "per_frame_calls_chained": {"value": job_throughput(tokens_per_step, args.steps, world, ms_next),
+                                    "unit": UNIT, "us_per_frame": 1e3 * ms_next / args.steps / w.frames,
+                                    "api": "hyb_attn_forward_next, one call per pass (the first pass of a "
+                                           "step through hyb_attn_forward)"},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "device_status": G.hyb_attn_status_string(status),

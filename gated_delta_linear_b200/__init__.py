@@ -26,6 +26,7 @@ from ._binding import (  # noqa: F401
     hyb_attn_workspace_bytes,
     hyb_attn_forward,
     hyb_attn_forward_branches,
+    hyb_attn_forward_next,
     hyb_attn_forward_noalloc,
     HYB_NOALLOC_SCRATCH_BYTES,
     hyb_attn_get_device_status,

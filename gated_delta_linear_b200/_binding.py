@@ -60,6 +60,8 @@ def _load():
     L.hyb_attn_workspace_bytes.restype = sz
     L.hyb_attn_forward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
     L.hyb_attn_forward.restype = i
+    L.hyb_attn_forward_next.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
+    L.hyb_attn_forward_next.restype = i
     L.hyb_attn_forward_branches.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp,
                                             vp, vp, vp, sz, vp]
     L.hyb_attn_forward_branches.restype = i
@@ -259,6 +261,17 @@ def hyb_attn_kernel_name(kernel: int):
     n = lib.hyb_attn_kernel_name(int(kernel))
     return n.decode() if n is not None else None
 
+def hyb_attn_forward_next(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state,
+                          clean_pass, out, workspace, workspace_bytes=None, stream=None) -> int:
+    """hyb_attn_forward continuing the chain of passes on ``workspace`` (the
+    next frame's W comes from the previous clean pass's update)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return lib.hyb_attn_forward_next(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(phi_q),
+                                     _ptr(phi_k), _ptr(phi_v), _ptr(gate_logits), _ptr(beta_logits),
+                                     _ptr(state), int(clean_pass), _ptr(out), _ptr(workspace),
+                                     workspace_bytes, _stream(stream))
+
 
 class HybridAttention:
     """Owns the device buffers of one layer instance and drives its passes.
@@ -290,6 +303,18 @@ class HybridAttention:
                               self.state, clean_pass, out, self.workspace, stream=stream)
         if st != HYB_OK:
             raise HybAttnError(st, "hyb_attn_forward")
+        return out
+
+    def forward_next(self, q, k, v, gate_logits, beta_logits, clean_pass, out=None, stream=None):
+        """``forward`` through hyb_attn_forward_next: consecutive calls on this
+        layer continue one chain (call ``forward`` after resetting the state)."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        st = hyb_attn_forward_next(self.desc, q, k, v, *self.phi, gate_logits, beta_logits,
+                                   self.state, clean_pass, out, self.workspace, stream=stream)
+        if st != HYB_OK:
+            raise HybAttnError(st, "hyb_attn_forward_next")
         return out
 
     def forward_branches(self, q, k, v, gate_logits, beta_logits, clean_pass, stream=None):

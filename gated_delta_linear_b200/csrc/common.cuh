@@ -45,6 +45,15 @@ struct LayerArgs {
     float* partials;           // fp32 [BH][nsplit][D][2D]: per-split [G | P]
     int nsplit;
     int split_tokens;
+    // chained passes (tensor path): the delta update lets the next kernel of the
+    // stream start at once (chain_trigger); before reading S_{N-1} it waits until
+    // the words chain_flags[bh * 8 + c], c < nsplit, equal chain_wait (0: no wait),
+    // which the previous chained update of this state sets once it is done with
+    // the state and its W; it sets its own words to chain_set (NULL: no flags)
+    unsigned* chain_flags;
+    unsigned chain_wait;
+    unsigned chain_set;
+    int chain_trigger;
     // token-level access: the inter-frame read computed by the token-level kernels,
     // fp32 [B][T][H][D]; the attention kernels add it instead of Q W (NULL: Q W)
     const float* oi_ext;

@@ -29,7 +29,7 @@ struct Plan {
     bool bf16;
     int nsplit;
     int split_tokens;
-    size_t off_W, off_Sprev, off_part, total;
+    size_t off_W, off_Sprev, off_part, off_chain, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -73,11 +73,15 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     update_split(d->T, bf16 ? third : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
     const size_t hh = (size_t)BH * D * D;
     p->off_W = kStatusBytes;
-    p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);   // fp32 W or two bf16 halves
+    // fp32 W, or the two bf16 halves of W; then the fp32 path's copy of S_{N-1},
+    // which on the tensor path is the second W slot of chained passes
+    p->off_Sprev = align_up(p->off_W + hh * sizeof(float), 256);
     p->off_part = align_up(p->off_Sprev + hh * sizeof(float), 256);
     // fp32 path: split partials (the tensor path reduces its splits on chip)
     const size_t part_bytes = bf16 ? 0 : hh * 2 * p->nsplit * sizeof(float);
-    p->total = align_up(p->off_part + part_bytes, 256);
+    // chained passes: one flag word per update CTA (a cluster of at most 8 per head)
+    p->off_chain = align_up(p->off_part + part_bytes, 256);
+    p->total = align_up(p->off_chain + (size_t)BH * tc::kMaxClusterRanks * sizeof(unsigned), 256);
     return HYB_OK;
 }
 
@@ -345,8 +349,59 @@ cudaError_t launch_tc(const LayerArgs& a, int clean, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// ---- chained passes -----------------------------------------------------------
+// What hyb_attn_forward_next knows about a workspace after its last pass there:
+// the pass's buffers and stream, the W slot that holds phi_q^T of the present
+// state, and the flag value the last chained delta update on this state sets
+// (0: none since the chain's prep).  Any other pass on the workspace or the
+// state drops the record, so the next chained call starts over with prep.
+struct ChainRec {
+    const void* ws = nullptr;  // null: free entry
+    const float* state;
+    const void* phi_q;
+    cudaStream_t stream;
+    int B, H, T, dtype, d;
+    float sm_scale, l2_eps;
+    int cur;
+    unsigned epoch;
+};
+constexpr int kChainRecs = 16;
+ChainRec g_chain[kChainRecs];
+unsigned g_chain_epoch = 0;
+int g_chain_victim = 0;
+
+void chain_forget(const void* ws, const float* state) {
+    for (ChainRec& r : g_chain)
+        if (r.ws && (r.ws == ws || (state && r.state == state))) r.ws = nullptr;
+}
+
+bool chain_find(const void* ws, ChainRec* out) {
+    for (const ChainRec& r : g_chain)
+        if (r.ws && r.ws == ws) {
+            *out = r;
+            return true;
+        }
+    return false;
+}
+
+void chain_store(const ChainRec& rec) {
+    for (ChainRec& r : g_chain)
+        if (!r.ws) {
+            r = rec;
+            return;
+        }
+    g_chain[g_chain_victim] = rec;
+    g_chain_victim = (g_chain_victim + 1) % kChainRecs;
+}
+
+unsigned chain_next_epoch() {
+    if (++g_chain_epoch == 0) ++g_chain_epoch;
+    return g_chain_epoch;
+}
+
 // Checks every argument of a pass and fills the kernels' argument block;
-// enqueues nothing, so an error here leaves the stream untouched.
+// enqueues nothing, so an error here leaves the stream untouched.  A pass on a
+// workspace or a state ends any chain of passes that used them.
 hyb_status pass_args(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
                      const void* phi_q, const void* phi_k, const void* phi_v, const float* gate_logits,
                      const float* beta_logits, float* state, int clean_pass, void* out, float* out_intra,
@@ -365,6 +420,7 @@ hyb_status pass_args(const hyb_attn_desc* desc, const void* q, const void* k, co
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return HYB_ERR_ALIGN;
     if (!workspace || workspace_bytes < p.total) return HYB_ERR_WORKSPACE;
+    chain_forget(workspace, state);
 
     LayerArgs a;
     memset(&a, 0, sizeof(a));
@@ -587,6 +643,7 @@ hyb_status kvcache_impl(const hyb_attn_desc* desc, const void* q, const void* k,
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return HYB_ERR_ALIGN;
     if (!workspace || workspace_bytes < kStatusBytes) return HYB_ERR_WORKSPACE;
+    chain_forget(workspace, nullptr);
 
     constexpr int D = 128;
     const int B = desc->B, H = desc->H, T = desc->T;
@@ -686,6 +743,67 @@ hyb_status hyb_attn_forward_mixed(const hyb_attn_desc* desc, const void* q, cons
     if (!mix || !out) return HYB_ERR_INVALID;
     return forward_impl(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass, out,
                         nullptr, nullptr, workspace, workspace_bytes, stream, mix);
+}
+
+hyb_status hyb_attn_forward_next(const hyb_attn_desc* desc, const void* q, const void* k, const void* v,
+                                 const void* phi_q, const void* phi_k, const void* phi_v,
+                                 const float* gate_logits, const float* beta_logits, float* state,
+                                 int clean_pass, void* out, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    if (!out) return HYB_ERR_INVALID;
+    ChainRec prev;
+    const bool had = chain_find(workspace, &prev);
+    LayerArgs a;
+    Plan p;
+    hyb_status s = pass_args(desc, q, k, v, phi_q, phi_k, phi_v, gate_logits, beta_logits, state, clean_pass,
+                             out, nullptr, nullptr, workspace, workspace_bytes, nullptr, &a, &p);
+    if (s != HYB_OK) return s;
+    if (!p.bf16) return launch_pass(a, p, clean_pass, stream);  // the fp32 path keeps no chain
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool cont = had && prev.state == state && prev.phi_q == phi_q && prev.stream == st &&
+                      prev.B == desc->B && prev.H == desc->H && prev.T == desc->T && prev.dtype == desc->dtype &&
+                      prev.d == desc->d_k && prev.sm_scale == desc->sm_scale && prev.l2_eps == desc->l2_eps;
+    // W slots: the pass reads slot `cur` and its delta update writes the other,
+    // which the attention kernel of this pass does not read
+    char* ws = (char*)workspace;
+    const size_t hh = (size_t)desc->B * desc->H * 128 * 128;
+    __nv_bfloat16* slot[2] = {(__nv_bfloat16*)(ws + p.off_W), (__nv_bfloat16*)(ws + p.off_Sprev)};
+    const int cur = cont ? prev.cur : 0;
+    unsigned epoch = cont ? prev.epoch : 0;
+    a.WT_hi = slot[cur];
+    a.WT_lo = a.WT_hi + hh;
+    if (clean_pass) {
+        a.w_next = slot[1 - cur];
+        a.chain_flags = (unsigned*)(ws + p.off_chain);
+        a.chain_wait = epoch;
+        a.chain_set = epoch = chain_next_epoch();
+        a.chain_trigger = 1;
+    }
+    TcPass tp;
+    cudaError_t e = tp.init(a);
+    // a continued chain has W of the present state in slot `cur` already (the
+    // previous clean pass's update wrote it, or a prep before a query-only pass)
+    if (e == cudaSuccess && !cont) e = tp.prep(st, true);
+    if (e == cudaSuccess) e = tp.attn(st, true);
+    if (e == cudaSuccess && clean_pass) e = tp.update(st, true);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return HYB_ERR_CUDA;
+    ChainRec rec;
+    rec.ws = workspace;
+    rec.state = state;
+    rec.phi_q = phi_q;
+    rec.stream = st;
+    rec.B = desc->B;
+    rec.H = desc->H;
+    rec.T = desc->T;
+    rec.dtype = desc->dtype;
+    rec.d = desc->d_k;
+    rec.sm_scale = desc->sm_scale;
+    rec.l2_eps = desc->l2_eps;
+    rec.cur = clean_pass ? 1 - cur : cur;
+    rec.epoch = epoch;
+    chain_store(rec);
+    return HYB_OK;
 }
 
 // ---- Token Radius Attention ------------------------------------------------------

@@ -108,6 +108,35 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// orders this thread's earlier generic-proxy accesses before its later
+// async-proxy ones (and the reverse), in every state space
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+
+// ------------------------------------------------------------------ flags between grids
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Waits until p[0..n) all equal `want` (acquire loads).  Bounded like mbar_wait:
+// after limit_ns it sets the workspace's TIMEOUT flag and returns false.
+__device__ __forceinline__ bool flags_wait_equal(const unsigned* p, int n, unsigned want, unsigned* gflags,
+                                                 uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    for (int c = 0; c < n; ++c) {
+        while (ld_acquire_gpu(p + c) != want) {
+            if (globaltimer_ns() - t0 > limit_ns) {
+                atomicOr(gflags, FLAG_TIMEOUT);
+                return false;
+            }
+            __nanosleep(128);
+        }
+    }
+    return true;
+}
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }

@@ -149,6 +149,10 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         if (threadIdx.x == 0) atomicOr(a.flags, FLAG_INTERNAL);
         return;
     }
+    // a chained pass: the next kernel of the stream (the next pass's attention,
+    // which reads W of the next frame only after this grid completes) may start
+    // on the SMs this grid leaves idle
+    if (a.chain_trigger) pdl_launch_dependents();
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
@@ -358,8 +362,21 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     __syncthreads();  // every MMA of the tile loop has completed (or timed out)
     tc_fence_after();
     if (threadIdx.x == kLoadWarp * 32) {
-        mbar_expect_tx(&bars[B_PARK], 128 * 128 * 4);
-        bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
+        // a chained pass may have started before the previous chained update has
+        // written S_{N-1}: wait for its flags (every CTA of its cluster raises one
+        // once it is done with the state), then read the state through the async proxy
+        bool chain_ok = true;
+        if (a.chain_wait) {
+            chain_ok = flags_wait_equal(a.chain_flags + (size_t)bh * kMaxClusterRanks, C, a.chain_wait, a.flags,
+                                        a.wait_ns);
+            fence_proxy_async_all();
+        }
+        if (chain_ok) {
+            mbar_expect_tx(&bars[B_PARK], 128 * 128 * 4);
+            bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
+        } else {
+            *abort_word = 1;  // nothing in flight; every later wait of the CTA gives up
+        }
     }
     {
         // alpha: the entry loads, then any further logits (T > 8 x 320), each
@@ -624,6 +641,14 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     // only after it: later work in the stream (the next prep, which rewrites the
     // W the attention kernel reads) stays ordered after both
     pdl_wait_primary();
+    if (a.chain_flags) {
+        // this CTA is done with the state (its band written, S_N read for W) and
+        // the attention kernel before it has completed: release the next chained
+        // update, which overwrites both the state and the W slot that kernel read
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) st_release_gpu(a.chain_flags + (size_t)bh * kMaxClusterRanks + split, a.chain_set);
+    }
 }
 
 // ============================================================== prep: W = phi_q^T S_{N-1}

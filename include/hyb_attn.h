@@ -103,6 +103,33 @@ hyb_status hyb_attn_forward(const hyb_attn_desc* desc,
                             float* state, int clean_pass, void* out,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* hyb_attn_forward_next -- the same pass as hyb_attn_forward (same arguments,
+ * bit-identical outputs and state), for one call per pass in a stream of passes
+ * (autoregressive use: the next frame's inputs exist only after this frame).
+ * The inter-frame read needs W = phi_q^T S_{N-1} (ARL2 summary §2.1); a clean
+ * pass's delta update already holds S_N, so here it also writes the next
+ * frame's W (the prep kernel's operands and instruction sequence), and the next
+ * call continues from it: no prep kernel, and its attention kernel starts
+ * while this pass's update still runs.  A call continues the chain when the
+ * previous pass on this workspace was a hyb_attn_forward_next call with the same
+ * descriptor, state, phi_q and stream; any other call (or a pass of any other
+ * entry point on this workspace or state) starts a new chain, which runs the
+ * prep kernel first, exactly as hyb_attn_forward.
+ * Caller's contract while a chain runs: nothing but these calls writes the
+ * state, phi_q or the workspace.  A caller that resets or restores the state
+ * starts the next chain with a hyb_attn_forward call (or any other pass on
+ * that workspace), which ends the old chain; the library cannot see a write
+ * the caller makes itself.  The chained update releases the next one through
+ * flag words in the workspace (a bounded device wait: HYB_ERR_TIMEOUT after
+ * 2 s).  The chain record is kept on the host for up to 16 workspaces; not
+ * thread-safe.  The fp32 path keeps no chain (each call is hyb_attn_forward). */
+hyb_status hyb_attn_forward_next(const hyb_attn_desc* desc,
+                                 const void* q, const void* k, const void* v,
+                                 const void* phi_q, const void* phi_k, const void* phi_v,
+                                 const float* gate_logits, const float* beta_logits,
+                                 float* state, int clean_pass, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Same pass, also writing the two branches separately in fp32 (for parity
  * checks); out may be NULL, out_intra and out_inter may not. */
 hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
