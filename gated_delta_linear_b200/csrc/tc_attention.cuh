@@ -17,13 +17,16 @@
 // major: an MN-major B operand), so the inter-frame read lands in TMEM next to
 // the softmax accumulator and the epilogue writes out = O_intra + O_inter once.
 //   TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,384) O,
-//                 [384,448) Q, [448,512) P (bf16, two per 32-bit column: the
-//                 A operands of S = Q K^T and O += P V).  Q is copied from
-//                 shared memory into TMEM once; as soon as the softmax has S_j
-//                 in registers the MMA warp issues S_{j+2} into its buffer, so
-//                 scores run a tile ahead of the softmax, and the softmax loads
-//                 S_{j+1} while it hands P_j over.  With both MMA A operands in
-//                 TMEM only the B operand (K or V) is read from shared memory.
+//                 [384,448) P buffer 0, [448,512) P buffer 1 (bf16, two per
+//                 32-bit column: the A operand of O += P V).  S = Q K^T takes
+//                 both operands from shared memory.  As soon as the softmax has
+//                 S_j in registers the MMA warp issues S_{j+2} into its buffer,
+//                 so scores run a tile ahead of the softmax, and the softmax
+//                 loads S_{j+1} while it hands P_j over.  P_j goes to buffer
+//                 j & 1, so the softmax never waits for P_{j-1} V_{j-1}: the
+//                 value product of one tile runs while the next tile's P is
+//                 written, and the tensor pipe is not idle for the round trip
+//                 from one value product's completion to the next P.
 //   Softmax: exponents against a running offset (the first tile's row max),
 //                 moved only when a tile's partial sum over a half row leaves
 //                 [0, 2^63); all exponentials on the MUFU pipe.
@@ -62,7 +65,11 @@ constexpr int kSoftmaxThreads = 256;           // warps 0-7: rows 32(w&3)..+31, 
 constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadVWarp = 10;
 constexpr int kThreads = 352;
 enum { B_Q = 0, B_W = 1, B_OIDONE = 2, B_KFULL = 3, B_KEMPTY = 6, B_VFULL = 9, B_VEMPTY = 12, B_SFULL = 15,
-       B_SREAD = 17, B_QTM = 19, B_PFULL = 20, B_PVDONE = 21, B_COUNT = 22 };
+       B_SREAD = 17, B_PFULL = 19, B_PVDONE = 21, B_COUNT = 23 };
+// per P buffer j & 1: B_PFULL + (j & 1) (P_j written) and B_PVDONE + (j & 1)
+// (P_j V_j done).  A softmax warp may run a tile ahead of another, so P_{j+1}
+// must not arrive on P_j's barrier; it cannot run two ahead (P_{j+2} waits for
+// P_j V_j, which waits for every warp's P_j).
 static_assert(B_COUNT * 8 + 8 <= 256, "barrier block");
 }  // namespace attn
 
@@ -163,7 +170,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // before the block synchronises (the loads land on its own barriers)
         for (int i = 0; i < B_COUNT; ++i)
             mbar_init(&bars[i],
-                      (i == B_PFULL || i == B_QTM || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads : 1);
+                      (i == B_PFULL || i == B_PFULL + 1 || i == B_SREAD || i == B_SREAD + 1) ? kSoftmaxThreads
+                                                                                              : 1);
         *abort_word = 0;
         *epi_bad = 0;
         fence_mbar_init();
@@ -185,9 +193,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // S buffers 0 / 1, O, Q and P as bf16 pairs (the A operands of the score
-    // and value products)
-    const uint32_t tS0 = tmem, tO = tmem + 256, tQ = tmem + 384, tP = tmem + 448;
+    // S buffers 0 / 1, O, and P buffers 0 / 1 as bf16 pairs (P_j in buffer j & 1:
+    // the A operand of O += P_j V_j)
+    const uint32_t tS0 = tmem, tO = tmem + 256, tP = tmem + 384;
     const uint32_t tOI = tS0 + (n & 1) * 128;  // the S buffer the last tile does not use
 
     if (warp == kLoadVWarp) {
@@ -244,19 +252,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
-        // S_j = Q K_j^T into S buffer j&1 (A = Q from TMEM); S_{j+2} reuses the
-        // buffer as soon as the softmax has S_j in registers, so scores run a
-        // tile ahead.  O += P_j V_j once P_j is in TMEM.
+        // S_j = Q K_j^T into S buffer j&1 (both operands from shared memory);
+        // S_{j+2} reuses the buffer as soon as the softmax has S_j in registers,
+        // so scores run a tile ahead.  O += P_j V_j once P_j is in its TMEM
+        // buffer; the softmax writes P_{j+1} into the other buffer meanwhile.
         if (lane == 0) {
             constexpr uint32_t ID_KK = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_KMN = idesc_bf16(128, 128, 0, 1);
             // descriptors of the first K stage (K-major and, for W, MN-major) and of
             // the first V stage; a stage's descriptor is this plus its offset / 16
-            const uint64_t dK = kmajor_desc(sb + K0, 0), dW = mnmajor_desc(sb + K0, 0), dV = mnmajor_desc(sb + V0, 0);
+            const uint64_t dQ = kmajor_desc(sb + Q, 0), dK = kmajor_desc(sb + K0, 0), dW = mnmajor_desc(sb + K0, 0),
+                           dV = mnmajor_desc(sb + V0, 0);
             constexpr uint64_t kStage = kTileBytes >> 4;
-            // S_0 and S_1 take Q from shared memory (no wait for its copy into TMEM)
             bool ok = mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns);
-            bool q_in_tmem = false;
             for (int j = 0; j < 2 && j < n && ok; ++j) {
                 if (!(ok = mbar_wait(&bars[B_KFULL + j], 0, abort_word, a.flags, a.wait_ns))) break;
                 tc_fence_after();
@@ -271,11 +279,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 const int sbuf = j & 1;
                 if (j + 2 < n) {
                     const int ks = (j + 2) % kKStages;
-                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags, a.wait_ns))) break;
                     if (!(ok = mbar_wait(&bars[B_SREAD + sbuf], (j >> 1) & 1, abort_word, a.flags, a.wait_ns))) break;
                     if (!(ok = mbar_wait(&bars[B_KFULL + ks], ((j + 2) / kKStages) & 1, abort_word, a.flags, a.wait_ns))) break;
                     tc_fence_after();
-                    mma8_ts<false>(tS0 + sbuf * 128, tQ, dK + ks * kStage, ID_KK, 0);
+                    mma8_ss<false>(tS0 + sbuf * 128, dQ, dK + ks * kStage, ID_KK, 0);
                     mma_commit(&bars[B_SFULL + sbuf]);
                     mma_commit(&bars[B_KEMPTY + ks]);
                 }
@@ -283,22 +290,21 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     // O_inter = Q W_hi + Q W_lo into S buffer n&1 (free once the
                     // softmax has S_{n-2} in registers; unused when n == 1), run
                     // while the softmax works on the last two tiles
-                    if (!q_in_tmem && !(ok = q_in_tmem = mbar_wait(&bars[B_QTM], 0, abort_word, a.flags, a.wait_ns))) break;
                     if (n >= 2 &&
                         !(ok = mbar_wait(&bars[B_SREAD + (n & 1)], ((n - 2) >> 1) & 1, abort_word, a.flags, a.wait_ns)))
                         break;
                     if (!(ok = mbar_wait(&bars[B_W], 0, abort_word, a.flags, a.wait_ns))) break;
                     tc_fence_after();
-                    mma8_ts<true>(tOI, tQ, dW + wst_hi * kStage, ID_KMN, 0);
-                    mma8_ts<true>(tOI, tQ, dW + wst_lo * kStage, ID_KMN, 1);
+                    mma8_ss<true>(tOI, dQ, dW + wst_hi * kStage, ID_KMN, 0);
+                    mma8_ss<true>(tOI, dQ, dW + wst_lo * kStage, ID_KMN, 1);
                     mma_commit(&bars[B_OIDONE]);
                 }
                 const int vs = j % kVStages;
-                if (!(ok = mbar_wait(&bars[B_PFULL], j & 1, abort_word, a.flags, a.wait_ns))) break;
+                if (!(ok = mbar_wait(&bars[B_PFULL + (j & 1)], (j >> 1) & 1, abort_word, a.flags, a.wait_ns))) break;
                 if (!(ok = mbar_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_word, a.flags, a.wait_ns))) break;
                 tc_fence_after();
-                mma8_ts<true>(tO, tP, dV + vs * kStage, ID_KMN, j > 0);
-                mma_commit(&bars[B_PVDONE]);
+                mma8_ts<true>(tO, tP + (j & 1) * 64, dV + vs * kStage, ID_KMN, j > 0);
+                mma_commit(&bars[B_PVDONE + (j & 1)]);
                 mma_commit(&bars[B_VEMPTY + vs]);
             }
             // drain: every MMA issued so far completes before TMEM is released
@@ -341,24 +347,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         float m = 0.f, l = 0.f;
         float A = 0.f;  // kEnt: sum of p (y - m) over this half of the row
         float x[64];
-        // this half of Q row r (128B-swizzled in shared memory) into TMEM as bf16 pairs
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_Q], 0, abort_word, a.flags, a.wait_ns));
-        if (ok) {
-            uint32_t qv[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(smem + Q + hf * kHalf + sw128_offset(r, c));
-                qv[4 * c] = v.x;
-                qv[4 * c + 1] = v.y;
-                qv[4 * c + 2] = v.z;
-                qv[4 * c + 3] = v.w;
-            }
-            tmem_st32u(tQ + lrow + hf * 32, qv);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[B_QTM]);
-        }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags, a.wait_ns));
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], 0, abort_word, a.flags, a.wait_ns));
         if (ok) {
             tc_fence_after();
             tmem_ld32(tS0 + lrow + cs, x);
@@ -418,9 +407,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             // sum p (y - m) against the moved offset: f (A - dm l) (p scales by f)
             if (kEnt) A = fmaf(f, A - dm * l, At);
             l = fmaf(l, f, lt);
-            // the P buffer (and O) are free once P_{j-1} V_{j-1} is done
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE], (j - 1) & 1, abort_word, a.flags, a.wait_ns));
+            // P buffer j & 1 is free once P_{j-2} V_{j-2} is done; a rescale of O
+            // also waits for P_{j-1} V_{j-1}
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + (j & 1)], ((j - 2) >> 1) & 1, abort_word,
+                                                       a.flags, a.wait_ns));
+                if (!ok) continue;
+                tc_fence_after();
+            }
+            if (any_redo && j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PVDONE + ((j - 1) & 1)], ((j - 1) >> 1) & 1,
+                                                       abort_word, a.flags, a.wait_ns));
                 if (!ok) continue;
                 tc_fence_after();
             }
@@ -435,7 +432,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     tmem_st32(tO + lrow + cs + c, o);
                 }
             }
-            tmem_st32u(tP + lrow + hf * 32, pk);
+            tmem_st32u(tP + (j & 1) * 64 + lrow + hf * 32, pk);
             // this half of S_{j+1} into registers while P_j is being stored
             if (j + 1 < n) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + (s ^ 1)], ((j + 1) >> 1) & 1, abort_word,
@@ -449,11 +446,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            if (ok) mbar_arrive(&bars[B_PFULL]);
+            if (ok) mbar_arrive(&bars[B_PFULL + (j & 1)]);
         }
         // epilogue: out = O / l + O_inter for this half of the row
         if (ok) tmem_ld_wait();
-        bool e_ok = ok && mbar_wait(&bars[B_PVDONE], (n - 1) & 1, abort_word, a.flags, a.wait_ns);
+        bool e_ok = ok && mbar_wait(&bars[B_PVDONE + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_word, a.flags, a.wait_ns);
         e_ok = __all_sync(0xffffffffu, e_ok && (!inter || mbar_wait(&bars[B_OIDONE], 0, abort_word, a.flags, a.wait_ns)));
         // row sum over the two halves (slot parity n&1: its last readers passed
         // the pair barrier of tile n-1)

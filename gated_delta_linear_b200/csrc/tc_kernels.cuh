@@ -60,6 +60,15 @@ __device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
                     kk > 0 ? 1u : acc0);
 }
 
+// The same with A from shared memory too: a K-major tile with descriptor a0 + step(kk).
+template <bool kMnB>
+__device__ __forceinline__ void mma8_ss(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc, uint32_t acc0) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(d_tmem, a0 + kmajor_step(kk), b0 + (kMnB ? mnmajor_step(kk) : kmajor_step(kk)), idesc,
+                 kk > 0 ? 1u : acc0);
+}
+
 // Max of N scores (fmaxf: NaN entries are skipped).
 template <int N>
 __device__ __forceinline__ float row_max(const float* x) {
