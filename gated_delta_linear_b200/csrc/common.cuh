@@ -46,10 +46,12 @@ struct LayerArgs {
     int nsplit;
     int split_tokens;
     // chained passes (tensor path): the delta update lets the next kernel of the
-    // stream start at once (chain_trigger); before reading S_{N-1} it waits until
-    // the words chain_flags[bh * 8 + c], c < nsplit, equal chain_wait (0: no wait),
-    // which the previous chained update of this state sets once it is done with
-    // the state and its W; it sets its own words to chain_set (NULL: no flags)
+    // stream start at its entry (chain_trigger 1) or once its key tiles are done
+    // (chain_trigger 2: the next update of a chain of updates); before reading
+    // S_{N-1} it waits until the words chain_flags[bh * 8 + c], c < nsplit, equal
+    // chain_wait (0: no wait), which the previous chained update of this state
+    // sets once it is done with the state and its W; it sets its own words to
+    // chain_set (NULL: no flags)
     unsigned* chain_flags;
     unsigned chain_wait;
     unsigned chain_set;

@@ -929,12 +929,20 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
         delete[] args;
         return HYB_ERR_INVALID;
     }
+    unsigned prev_epoch = 0;
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
         args[n].WT_hi = (__nv_bfloat16*)(slots + n * wslot);
         args[n].WT_lo = args[n].WT_hi + hh;
         // the update of frame n also writes W of frame n + 1 (what prep would
         // compute from S_n), so the chain is one kernel per frame
         args[n].w_next = n + 1 < n_frames ? (__nv_bfloat16*)(slots + (n + 1) * wslot) : nullptr;
+        // consecutive updates overlap: update n + 1 starts (PDL) once every CTA
+        // of update n has finished its key tiles, walks its own, and waits for
+        // update n's flags before it reads S_n (at most two updates hold SMs)
+        args[n].chain_flags = (unsigned*)((char*)workspace + p.off_chain);
+        args[n].chain_wait = prev_epoch;
+        args[n].chain_set = prev_epoch = chain_next_epoch();
+        args[n].chain_trigger = 2;
         e = tp[n].init(args[n]);
     }
     if (e == cudaSuccess) e = cudaEventRecord(r->fork, st);
@@ -943,7 +951,7 @@ hyb_status hyb_attn_forward_frames(const hyb_attn_desc* desc, int n_frames, cons
     if (e == cudaSuccess) e = tp[0].prep(r->chain, false);
     if (e == cudaSuccess) e = cudaEventRecord(r->w[0], r->chain);
     for (int n = 0; n < n_frames && e == cudaSuccess; ++n) {
-        if ((e = tp[n].update(r->chain, false)) != cudaSuccess) break;
+        if ((e = tp[n].update(r->chain, n > 0)) != cudaSuccess) break;
         if (n + 1 < n_frames && (e = cudaEventRecord(r->w[n + 1], r->chain)) != cudaSuccess) break;
         cudaStream_t att = r->att[n % kAttStreams];
         if ((e = cudaStreamWaitEvent(att, r->w[n], 0)) != cudaSuccess) break;

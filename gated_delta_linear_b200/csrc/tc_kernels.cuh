@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     // a chained pass: the next kernel of the stream (the next pass's attention,
     // which reads W of the next frame only after this grid completes) may start
     // on the SMs this grid leaves idle
-    if (a.chain_trigger) pdl_launch_dependents();
+    if (a.chain_trigger == 1) pdl_launch_dependents();
     const uint32_t sb = smem_u32(smem);
     uint64_t* bars = (uint64_t*)(smem + BAR);
     uint32_t* tmem_slot = (uint32_t*)(bars + B_COUNT);
@@ -370,6 +370,9 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     tc_fence_before();
     __syncthreads();  // every MMA of the tile loop has completed (or timed out)
     tc_fence_after();
+    // the next update of a chain of updates (its key tiles need nothing from
+    // this one) may start once every CTA here has finished its key tiles
+    if (a.chain_trigger == 2) pdl_launch_dependents();
     if (threadIdx.x == kLoadWarp * 32) {
         // a chained pass may have started before the previous chained update has
         // written S_{N-1}: wait for its flags (every CTA of its cluster raises one
