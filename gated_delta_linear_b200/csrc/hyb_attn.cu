@@ -64,13 +64,14 @@ hyb_status make_plan(const hyb_attn_desc* d, Plan* p) {
     // Tensor path: one cluster of at most 8 CTAs per (b, h), splits reduced in
     // distributed shared memory (no partials in the workspace).  The update runs
     // beside attention kernels (the second wave of its own frame's, or the next
-    // frame's), so its splits take about a third of the SMs in all and at least 3
-    // per head: fewer CTAs per head cost less SM time for the same work, more
-    // shorten the chain from one frame's state to the next.  fp32 path: enough
-    // (b, h, split) blocks to cover the SMs, partials in the workspace.
+    // frame's), so its splits take about a quarter of the SMs in all and at least
+    // 3 per head: fewer CTAs per head cost less SM time for the same work, more
+    // shorten the chain from one frame's state to the next (which consecutive
+    // updates of a frames call overlap).  fp32 path: enough (b, h, split) blocks
+    // to cover the SMs, partials in the workspace.
     const int BH = d->B * d->H;
-    const int third = kNumSMs / (3 * BH) > 3 ? kNumSMs / (3 * BH) : 3;
-    update_split(d->T, bf16 ? third : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
+    const int quarter = kNumSMs / (4 * BH) > 3 ? kNumSMs / (4 * BH) : 3;
+    update_split(d->T, bf16 ? quarter : (kNumSMs + BH - 1) / BH, bf16, &p->nsplit, &p->split_tokens);
     const size_t hh = (size_t)BH * D * D;
     p->off_W = kStatusBytes;
     // fp32 W, or the two bf16 halves of W; then the fp32 path's copy of S_{N-1},
