@@ -147,7 +147,10 @@ hyb_status hyb_attn_forward_branches(const hyb_attn_desc* desc,
  * frame N's attention, so the call runs the short sequential chain (W_N, then
  * S_N, frame after frame) on one internal stream and the attention kernels on
  * two others, frame after frame in turn, each attention kernel waiting only for
- * its own W_N: the attention kernels of consecutive frames share the SMs.  The
+ * its own W_N: the attention kernels of consecutive frames share the SMs, and
+ * consecutive state updates overlap (the next walks its key tiles while the
+ * current one reduces and writes the state; flag words in the workspace order
+ * their accesses to the state, with a bounded device wait).  The
  * results are bit-identical to the loop: the same kernels with the same
  * arithmetic; only their scheduling differs (for the fp32 path the call is the
  * loop).  The internal streams (the chain's at the highest priority) and events
