@@ -373,6 +373,7 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     // the next update of a chain of updates (its key tiles need nothing from
     // this one) may start once every CTA here has finished its key tiles
     if (a.chain_trigger == 2) pdl_launch_dependents();
+    bool park_issued = false, wphi_issued = false;  // (loader) copies to drain before exit
     if (threadIdx.x == kLoadWarp * 32) {
         // a chained pass may have started before the previous chained update has
         // written S_{N-1}: wait for its flags (every CTA of its cluster raises one
@@ -386,6 +387,7 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         if (chain_ok) {
             mbar_expect_tx(&bars[B_PARK], 128 * 128 * 4);
             bulk_load(sb + SPREV, a.state + (size_t)bh * 128 * 128, 128 * 128 * 4, &bars[B_PARK]);
+            park_issued = true;
         } else {
             *abort_word = 1;  // nothing in flight; every later wait of the CTA gives up
         }
@@ -513,13 +515,14 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         for (int w = 0; w < kThreads / 32; ++w) t += wsum[w];
         wsum[10] = t / (float)T;
     }
-    if (a.w_next && threadIdx.x == kLoadWarp * 32) {
+    if (a.w_next && threadIdx.x == kLoadWarp * 32 && !*abort_word) {
         // the Delta products have completed: phi_q (for the next frame's W) into
         // the phi_v tile, as an MN-major A operand
         tma_prefetch_desc(&tm_phiq);
         mbar_expect_tx(&bars[B_WPHI], kTileBytes);
         tma_load_3d(sb + PHIV, &tm_phiq, &bars[B_WPHI], 0, 0, h);
         tma_load_3d(sb + PHIV + kHalf, &tm_phiq, &bars[B_WPHI], 64, 0, h);
+        wphi_issued = true;
     }
     cluster_sync();  // every CTA of the cluster has parked Delta_c and staged S_{N-1}
 
@@ -648,6 +651,9 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
         __syncthreads();
         tc_fence_after();
     }
+    // after a wait gave up, copies this CTA issued may still be landing
+    if (park_issued) mbar_drain(&bars[B_PARK], 0, a.wait_ns);
+    if (wphi_issued) mbar_drain(&bars[B_WPHI], 0, a.wait_ns);
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
     // when launched as a programmatic dependent of the attention kernel, complete
     // only after it: later work in the stream (the next prep, which rewrites the
