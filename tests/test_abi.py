@@ -95,6 +95,31 @@ def test_host_validation_rejects_before_launch():
     assert G.hyb_attn_get_device_status(FAKE + 4, 0) == G.HYB_ERR_ALIGN
 
 
+def test_chained_entry_point_validates_like_the_plain_one():
+    """hyb_attn_forward_next checks every argument before anything is enqueued,
+    with the statuses of hyb_attn_forward (no chain record is kept for a call
+    that fails its checks)."""
+    d = G.make_desc(1, 12, 1560, 128)
+
+    def nxt(desc=d, **over):
+        args = dict(q=FAKE, k=FAKE, v=FAKE, phi_q=FAKE, phi_k=FAKE, phi_v=FAKE, gate_logits=FAKE,
+                    beta_logits=FAKE, state=FAKE, clean_pass=1, out=FAKE, workspace=FAKE,
+                    workspace_bytes=1 << 40, stream=0)
+        args.update(over)
+        return G.hyb_attn_forward_next(desc, **args)
+
+    assert G.lib.hyb_attn_forward_next(None, *([None] * 9), 0, None, None, 0, None) == G.HYB_ERR_INVALID
+    assert nxt(desc=G.make_desc(1, 12, 1560, 64)) == G.HYB_ERR_UNSUPPORTED
+    assert nxt(q=None) == G.HYB_ERR_INVALID
+    assert nxt(out=None) == G.HYB_ERR_INVALID
+    assert nxt(gate_logits=None) == G.HYB_ERR_INVALID
+    assert nxt(clean_pass=2) == G.HYB_ERR_INVALID
+    assert nxt(v=FAKE + 2) == G.HYB_ERR_ALIGN
+    assert nxt(workspace=None) == G.HYB_ERR_WORKSPACE
+    need = G.hyb_attn_workspace_bytes(d)
+    assert nxt(workspace_bytes=need - 1) == G.HYB_ERR_WORKSPACE
+
+
 def test_desc_layout_matches_header():
     # eight 4-byte fields, in the header's order
     assert ctypes.sizeof(G.HybAttnDesc) == 32
