@@ -69,6 +69,8 @@ struct LayerArgs {
     // optional: CTA i of the grid takes query tile row kv_order[i] (bh * n_qt + qt),
     // so the longest lists go first
     const int* kv_order;
+    // attention: consecutive query tiles per CTA (0 or 1: one)
+    int q_per_cta;
     // bounded device waits give up after wait_ns (2 s unless a fault test shortens it)
     unsigned long long wait_ns;
     int dbg_skip_v;            // fault test only: the attention kernel's V producer issues nothing

@@ -145,6 +145,20 @@ cudaError_t opt_in_smem(K kernel, size_t bytes, unsigned char* done) {
 // CTAs of the attention kernel along the query axis: one per 128-query tile.
 unsigned attn_tiles(int T) { return (unsigned)((T + tc::kTile - 1) / tc::kTile); }
 
+// Query tiles per attention CTA for a chained pass: two when one tile per CTA
+// would take more than one wave of the SMs but at most two (the second nearly
+// empty for a 480p frame), so the grid fits one wave and leaves SMs to the delta
+// update that runs beside it; one otherwise, and for block-sparse and entropy
+// passes (whose CTAs take one listed tile each).  (A CTA runs its tiles one
+// after another, so an attention kernel alone gains nothing from this, and a
+// frames call, which packs consecutive frames' kernels, runs one tile per CTA.)
+int attn_q_per_cta(const LayerArgs& a) {
+    const long long tiles = (long long)attn_tiles(a.T) * a.H * a.B;
+    const int key_tiles = (a.T_kv + tc::kTile - 1) / tc::kTile;
+    if (a.kv_list || a.kv_order || a.ent_out || !a.inter || key_tiles < 3) return 1;
+    return tiles > kNumSMs && tiles <= 2 * kNumSMs ? 2 : 1;
+}
+
 template <int D, typename TIO>
 cudaError_t launch_simt(const LayerArgs& a, int clean, cudaStream_t st) {
     static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_part[kMaxDevices],
@@ -252,11 +266,14 @@ struct TcPass {
         static unsigned char done_prep[kMaxDevices], done_attn[kMaxDevices], done_upd[kMaxDevices];
         constexpr int D = 128;
         a = args;
+        a.q_per_cta = 1;
         cudaError_t e;
         if ((e = opt_in_smem(tc::prep_tc_kernel, tc::prep::SMEM, done_prep)) != cudaSuccess) return e;
-        static unsigned char done_attn_ent[kMaxDevices];
+        static unsigned char done_attn_ent[kMaxDevices], done_attn_multi[kMaxDevices];
         if ((e = opt_in_smem(tc::attention_kernel<false>, tc::attn::SMEM, done_attn)) != cudaSuccess) return e;
         if ((e = opt_in_smem(tc::attention_kernel<true>, tc::attn::SMEM, done_attn_ent)) != cudaSuccess) return e;
+        if ((e = opt_in_smem(tc::attention_kernel<false, true>, tc::attn::SMEM, done_attn_multi)) != cudaSuccess)
+            return e;
         if ((e = opt_in_smem(tc::update_kernel, tc::upd::SMEM, done_upd)) != cudaSuccess) return e;
         const uint64_t row_bytes = (uint64_t)a.H * D * 2;
         const uint64_t bh = (uint64_t)a.B * a.H;
@@ -296,7 +313,8 @@ struct TcPass {
         cudaLaunchAttribute at[1];
         pdl_attr(&at[0]);
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(attn_tiles(a.T), a.H, a.B);
+        const unsigned qpc = a.q_per_cta > 1 ? (unsigned)a.q_per_cta : 1u;
+        cfg.gridDim = dim3((attn_tiles(a.T) + qpc - 1) / qpc, a.H, a.B);
         cfg.blockDim = dim3(tc::attn::kThreads, 1, 1);
         cfg.dynamicSmemBytes = tc::attn::SMEM;
         cfg.stream = st;
@@ -305,8 +323,9 @@ struct TcPass {
         cudaError_t le = cudaSuccess;
         // the entropy-writing variant for the warm-up pass of Token Radius Attention
         cudaError_t e = timed(K_ATTN, st, [&] {
-            le = a.ent_out ? cudaLaunchKernelEx(&cfg, tc::attention_kernel<true>, a, tq, tk, tv, tw, tout)
-                           : cudaLaunchKernelEx(&cfg, tc::attention_kernel<false>, a, tq, tk, tv, tw, tout);
+            le = a.ent_out       ? cudaLaunchKernelEx(&cfg, tc::attention_kernel<true>, a, tq, tk, tv, tw, tout)
+                 : qpc > 1       ? cudaLaunchKernelEx(&cfg, tc::attention_kernel<false, true>, a, tq, tk, tv, tw, tout)
+                                 : cudaLaunchKernelEx(&cfg, tc::attention_kernel<false>, a, tq, tk, tv, tw, tout);
         });
         return e != cudaSuccess ? e : le;
     }
@@ -782,6 +801,7 @@ hyb_status hyb_attn_forward_next(const hyb_attn_desc* desc, const void* q, const
     }
     TcPass tp;
     cudaError_t e = tp.init(a);
+    tp.a.q_per_cta = attn_q_per_cta(tp.a);
     // a continued chain has W of the present state in slot `cur` already (the
     // previous clean pass's update wrote it, or a prep before a query-only pass)
     if (e == cudaSuccess && !cont) e = tp.prep(st, true);
