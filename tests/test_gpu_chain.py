@@ -97,6 +97,14 @@ def test_chain_ragged_length_matches_oracle():
 
 
 @pytest.mark.gpu
+def test_chain_two_query_tiles_per_cta_ragged_matches_oracle():
+    # 12 heads x 13 query tiles (the last holding one row): chained passes run
+    # two consecutive query tiles per attention CTA, 7 CTAs per head, the last
+    # with one tile
+    _compare(W.small_workload(W.WORKLOADS[1], T=1537, frames=3), check_oracle=True)
+
+
+@pytest.mark.gpu
 def test_chain_streaming_passes_equal_loop():
     # 4 query-only passes and a clean pass per frame on a pre-filled state
     _compare(W.small_workload(W.WORKLOADS[2], H=12, frames=3, prior_frames=4))
