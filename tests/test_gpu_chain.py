@@ -201,3 +201,37 @@ def test_chain_other_stream_starts_a_new_chain():
         assert torch.equal(a, b)
     assert torch.equal(ref_s, s)
     assert G.hyb_attn_get_device_status(ws) == G.HYB_OK
+
+
+@pytest.mark.gpu
+def test_chain_interleaved_with_a_frames_call():
+    """Chained passes, then a frames call on the same state and workspace (it
+    ends the chain and writes the state), then chained passes again: every
+    output and the final state equal the per-pass loop of hyb_attn_forward."""
+    w = W.small_workload(W.WORKLOADS[1], H=4, T=300, frames=9)
+    G, phi, desc, passes, xs, dev = _setup(w)
+    s0 = torch.zeros(w.B, w.H, w.d, w.d, dtype=torch.float32, device="cuda")
+    ref_o, ref_s, _ = _run(G, G.hyb_attn_forward, desc, phi, passes, dev, s0)
+    nb = G.hyb_attn_frames_workspace_bytes(desc, 3)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    s = s0.clone()
+    outs = []
+    for i in range(3):
+        q, k, v, g, b = dev[i]
+        o = torch.empty_like(q)
+        assert G.hyb_attn_forward_next(desc, q, k, v, *phi, g, b, s, 1, o, ws) == G.HYB_OK
+        outs.append(o)
+    stk = [torch.stack([dev[i][f] for i in range(3, 6)]).contiguous() for f in range(5)]
+    of = torch.empty_like(stk[0])
+    assert G.hyb_attn_forward_frames(desc, 3, *stk[:3], *phi, *stk[3:], s, of, ws) == G.HYB_OK
+    outs += [of[i] for i in range(3)]
+    for i in range(6, 9):
+        q, k, v, g, b = dev[i]
+        o = torch.empty_like(q)
+        assert G.hyb_attn_forward_next(desc, q, k, v, *phi, g, b, s, 1, o, ws) == G.HYB_OK
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert G.hyb_attn_get_device_status(ws) == G.HYB_OK
+    for i, (a, b) in enumerate(zip(ref_o, outs)):
+        assert torch.equal(a, b), f"pass {i}"
+    assert torch.equal(ref_s, s)
