@@ -8,7 +8,9 @@
 // every token reads the same pre-update state).  The layer output is
 // O_intra + O_inter (the pages leave the combination open; this library sums).
 //
-// attention_kernel: one CTA per (128-query tile, head, batch), 11 warps.
+// attention_kernel: one CTA per (128-query tile, head, batch), 11 warps (the
+// kMulti variant: per run of consecutive query tiles of a head, taken one after
+// another, each as below).
 // Warp 8 streams Q and the K ring, warp 10 the V ring, with TMA into
 // 128B-swizzled shared memory; warp 9 issues the tcgen05 MMAs; warps 0-7 run
 // the online softmax, a query row per pair of threads (warps w and w+4, 64
