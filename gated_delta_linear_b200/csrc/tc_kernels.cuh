@@ -116,7 +116,7 @@ constexpr int kNormThreads = 256;                         // warps 0-7
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = 320;
 enum { B_PHI = 0, B_KFULL, B_KFREE, B_VFULL, B_KTFULL, B_KTFULL1, B_KTREAD, B_KTREAD1, B_OPSFULL, B_OPSFREE,
-       B_PARK, B_DELTA, B_WPHI, B_WMMA, B_COUNT };
+       B_PARK, B_DELTA, B_WPHI, B_WMMA, B_DRAIN, B_COUNT };
 static_assert(RED + 128 * 128 * 4 <= TILES_END, "post-loop buffers exceed the tile space");
 // byte offset of float4 chunk q (0..31) of row `row` in RED
 __device__ __forceinline__ uint32_t red_off(int row, int q) {
@@ -654,7 +654,16 @@ __global__ void __launch_bounds__(upd::kThreads, 1)
     // after a wait gave up, copies this CTA issued may still be landing
     if (park_issued) mbar_drain(&bars[B_PARK], 0, a.wait_ns);
     if (wphi_issued) mbar_drain(&bars[B_WPHI], 0, a.wait_ns);
-    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) {
+        // every product this CTA issued completes before its TMEM is released
+        // (after a wait gave up, some were issued without being waited for)
+        if (lane == 0) {
+            mma_commit(&bars[B_DRAIN]);
+            mbar_drain(&bars[B_DRAIN], 0, a.wait_ns);
+        }
+        __syncwarp();
+        tmem_dealloc(tmem, 512);
+    }
     // when launched as a programmatic dependent of the attention kernel, complete
     // only after it: later work in the stream (the next prep, which rewrites the
     // W the attention kernel reads) stays ordered after both
