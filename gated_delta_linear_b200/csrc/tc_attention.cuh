@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const uint32_t tS0 = tmem, tO = tmem + 256, tP = tmem + 384;
     // O_inter of tile t: the S buffer its last key tile does not use
     auto tOI_of = [&](int base) { return tS0 + ((base + n) & 1) * 128; };
+    // (producers) the last step whose V / K tile was issued (the first K tiles at
+    // entry), the last query tile whose Q and W were issued: after a wait gave
+    // up, these loads may still be landing when the block ends
+    int vg_last = -1, kg_last = (n < kKStages ? n : kKStages) - 1, q_last = 0, w_last = -1;
 
     if (warp == kLoadVWarp) {
         // ------------------------------------------------ TMA producer: V ring
@@ -226,7 +230,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                 mbar_expect_tx(&bars[B_VFULL + vs], kTileBytes);
                 tma_load_3d(sb + V0 + vs * kTileBytes, &tm_v, &bars[B_VFULL + vs], xh, kt * kTile, b);
                 tma_load_3d(sb + V0 + vs * kTileBytes + kHalf, &tm_v, &bars[B_VFULL + vs], xh + 64, kt * kTile, b);
+                vg_last = g;
             }
+
         }
         __syncwarp();
     } else if (warp == kLoadWarp) {
@@ -248,6 +254,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     mbar_expect_tx(&bars[B_Q], kTileBytes);
                     tma_load_3d(sb + Q, &tm_q, &bars[B_Q], xh, q0_of(t), b);
                     tma_load_3d(sb + Q + kHalf, &tm_q, &bars[B_Q], xh + 64, q0_of(t), b);
+                    q_last = t;
                     if (inter && !(ok = mbar_wait(&bars[B_OIDONE], (t - 1) & 1, abort_word, a.flags, a.wait_ns)))
                         break;
                 }
@@ -261,6 +268,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     tma_load_3d(sb + K0 + ks * kTileBytes, &tm_k, &bars[B_KFULL + ks], xh, ktile(j) * kTile, b);
                     tma_load_3d(sb + K0 + ks * kTileBytes + kHalf, &tm_k, &bars[B_KFULL + ks], xh + 64,
                                 ktile(j) * kTile, b);
+                    kg_last = g;
                 }
                 // W_hi / W_lo (row-major, MN-major operands) into K stages freed by
                 // S_{n-3} / S_{n-2} of this tile
@@ -280,8 +288,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                     tma_load_3d(sb + K0 + wst_hi * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, bh);
                     tma_load_3d(sb + K0 + wst_lo * kTileBytes, &tm_w, &bars[B_W], 0, 0, nbh + bh);
                     tma_load_3d(sb + K0 + wst_lo * kTileBytes + kHalf, &tm_w, &bars[B_W], 64, 0, nbh + bh);
+                    w_last = t;
                 }
             }
+
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -656,6 +666,19 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // every load a producer issued has landed before the block ends (in a normal
+    // run each phase below has long completed; after a wait gave up, some loads
+    // were never waited for): the last one on each barrier, bounded (no later
+    // load completes a phase of the same barrier)
+    if (threadIdx.x == kLoadVWarp * 32) {
+        for (int g = vg_last >= kVStages ? vg_last - kVStages + 1 : 0; g <= vg_last; ++g)
+            mbar_drain(&bars[B_VFULL + g % kVStages], (g / kVStages) & 1, a.wait_ns);
+    } else if (threadIdx.x == kLoadWarp * 32) {
+        for (int g = kg_last >= kKStages ? kg_last - kKStages + 1 : 0; g <= kg_last; ++g)
+            mbar_drain(&bars[B_KFULL + g % kKStages], (g / kKStages) & 1, a.wait_ns);
+        mbar_drain(&bars[B_Q], q_last & 1, a.wait_ns);
+        if (w_last >= 0) mbar_drain(&bars[B_W], w_last & 1, a.wait_ns);
+    }
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
