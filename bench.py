@@ -161,8 +161,10 @@ def run_reference(args):
         return 0
     import workloads as W
     w = W.WORKLOADS[WORKLOAD_ID]
-    # one step = one frame of the workload (all heads, one clean pass), oracle as it stands
-    oracle_frames(w, 1e9, max_frames=args.warmup)
+    # one step = one frame of the workload (all heads, one clean pass), oracle as it
+    # stands; at least 3 untimed warm-up frames, as for the CUDA arm
+    warmup = max(3, args.warmup)
+    oracle_frames(w, 1e9, max_frames=warmup)
     times = []
     for _ in range(args.steps):
         n, s = oracle_frames(w, 1e9, max_frames=1)
@@ -172,7 +174,7 @@ def run_reference(args):
     sample = f"{args.steps} frames (1 step = 1 frame, all {w.H} heads, float64 NumPy oracle)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(w, {"step": "one frame"}),
